@@ -1,0 +1,380 @@
+#!/usr/bin/env python
+"""Benchmark of the PISA prefill hot path on B200.
+
+One step = mean-pooled key pyramid + PISA top-K selection + block-sparse
+attention over one full synthetic input (default: 262144 tokens, 16 query
+heads, 2 kv heads, d = 128, C = 64, K = 16, bf16, causal, 256 planted
+needles). The flat single-level selector and the decode step (64 sequences x
+131072 cached tokens) are timed beside it and reported in the same line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun each rank runs the same workload on its own GPU (weak
+scaling: the path shards over independent sequences and heads with no
+collective); the barrier-bracketed time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hierarchical_top_block_mean_b200 import api, workloads  # noqa: E402
+
+METRIC = "PISA prefill tokens/s (select+attn) at 64K/256K; decode select µs/step"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def dist_init(n_gpus):
+    if n_gpus > 1 or "RANK" in os.environ:
+        import torch.distributed as dist
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+        return dist
+    return None
+
+
+def max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    dev = torch.device("cuda") if torch.cuda.is_available() else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+# -------------------------------------------------------------- algorithmic models
+
+def attn_bytes(w) -> float:
+    """Bytes the sparse attention must move per launch: q and out once, plus
+    the K and V rows of each row's selected blocks (per kv head and query:
+    K blocks of C keys, causally clipped), with no reuse across queries."""
+    e = 2 if w.dtype == "bf16" else 4
+    qo = 2 * w.B * w.H_q * w.N * w.d * e
+    keys = 0
+    for t in range(0, w.N, max(1, w.N // 4096)):
+        keys += min(w.K * w.C, t + 1)
+    keys *= w.N / len(range(0, w.N, max(1, w.N // 4096)))
+    return qo + 2 * w.B * w.H_kv * keys * w.d * e
+
+
+def pyramid_bytes(w) -> float:
+    e = 2 if w.dtype == "bf16" else 4
+    R = api.pyramid_rows(w.N, w.C)
+    return w.B * w.H_kv * (w.N * w.d * e + R * w.d * 4)
+
+
+# ------------------------------------------------------------------ arms
+
+def cpu_baseline(w, x, budget_s=15.0):
+    """The fp64 CPU oracle as it stands, on a bounded sample: the full
+    pyramid plus select + attention for a seeded sample of rows, scaled to
+    tokens/s over all rows."""
+    import numpy as np
+    import oracle as O
+    O.build()
+    cores = len(os.sched_getaffinity(0))
+    qh, kh, vh = (x[n].detach().cpu().contiguous() for n in ("q", "k", "v"))
+    cfg = O.make_cfg(B=w.B, N=w.N, H_q=w.H_q, H_kv=w.H_kv, d=w.d, C=w.C, K=w.K, causal=w.causal,
+                     dtype_code=0 if w.dtype == "f32" else 1)
+    t0 = time.perf_counter()
+    pyr = O.build_pyramid(kh, w.C)
+    t_pyr = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    n_rows, t_rows = 0, 0.0
+    batch = 64
+    while t_rows < budget_s and n_rows < w.B * w.H_kv * w.N:
+        ts = rng.integers(0, w.N, batch)
+        hs = rng.integers(0, w.H_kv, batch)
+        rows = np.stack([np.zeros(batch, np.int64), hs, ts], 1)
+        t1 = time.perf_counter()
+        sel, _ = O.select_rows(cfg, qh, kh, pyr, rows)
+        O.attn_rows(cfg, qh, kh, vh, rows, sel)
+        t_rows += time.perf_counter() - t1
+        n_rows += batch
+    total_rows = w.B * w.H_kv * w.N
+    est = t_pyr + t_rows * total_rows / n_rows
+    return {"value": w.B * w.N / est, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle: full pyramid ({t_pyr:.1f} s) + select+attention on {n_rows} random "
+                      f"(kv head, query) rows ({t_rows:.1f} s), extrapolated linearly to all {total_rows} rows"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle as it stands, timed on the host cores."""
+    dist = dist_init(args.gpus)
+    rank = dist.get_rank() if dist else 0
+    if rank != 0:
+        return 0
+    w = workloads.PREFILL[args.workload]
+    x = workloads.prefill_inputs(w, device="cpu")
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(w, x, budget_s=budget)
+    vals = [cpu_baseline(w, x, budget_s=budget) for _ in range(args.steps)]
+    v = statistics.median(r["value"] for r in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.B * w.N / v * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "C": w.C,
+                       "K": w.K, "causal": w.causal, "input_dtype": w.dtype},
+            "cpu_baseline": dict(vals[-1], value=v),
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+def time_decode(wd, steps=32, warmup=4):
+    """µs per decode step (append + fused select + attention) on the decode workload."""
+    dev = torch.device("cuda")
+    kc, vc, lens = workloads.decode_cache(wd, device=dev)
+    st = api.DecodeState(S=wd.S, cap=wd.cap, H_q=wd.H_q, H_kv=wd.H_kv, d=wd.d, C=wd.C, K=wd.K,
+                         dtype=wd.torch_dtype, device=dev, k_cache=kc, v_cache=vc, lens=lens)
+    st.init()
+    ins = [workloads.decode_step_inputs(wd, s, device=dev) for s in range(steps + warmup)]
+    for s in range(warmup):
+        st.step(*ins[s], keep_sel=False)
+    e0, e1 = events(2)
+    torch.cuda.synchronize()
+    e0.record()
+    for s in range(warmup, warmup + steps):
+        st.step(*ins[s], keep_sel=False)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / steps
+    # Selection alone on the same state.
+    q = ins[0][0]
+    e0.record()
+    for _ in range(steps):
+        st.select(q)
+    e1.record()
+    torch.cuda.synchronize()
+    us_sel = e0.elapsed_time(e1) * 1e3 / steps
+    ok = int(st.status.item()) == 0
+    del st, kc, vc
+    torch.cuda.empty_cache()
+    return {"workload": wd.name, "us_per_step": us, "select_us": us_sel, "steps": steps, "status_ok": ok}
+
+
+def run_gpu(args):
+    dist = dist_init(args.gpus)
+    rank = dist.get_rank() if dist else 0
+    world = dist.get_world_size() if dist else 1
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workloads.PREFILL[args.workload]
+    x = workloads.prefill_inputs(w, device=dev)
+    q, k, v = x["q"], x["k"], x["v"]
+    pr = api.Problem.of(q, k, C=w.C, K=w.K, causal=w.causal)
+    p = api.Prefill(pr, dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        p(q, k, v)
+    torch.cuda.synchronize()
+
+    n_ev = 4
+    evs = [events(n_ev) for _ in range(args.steps)]
+    launches0 = api.launch_count()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0 = time.perf_counter()
+        for s in range(args.steps):
+            e = evs[s]
+            e[0].record(stream)
+            p.pyramid(k)
+            e[1].record(stream)
+            p.select(q, k)
+            e[2].record(stream)
+            p.attend(q, k, v)
+            e[3].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+        if dist:
+            dist.barrier()
+    launches = api.launch_count() - launches0
+    stage = {"pyramid": 0.0, "select": 0.0, "attn": 0.0}
+    for e in evs:
+        stage["pyramid"] += e[0].elapsed_time(e[1])
+        stage["select"] += e[1].elapsed_time(e[2])
+        stage["attn"] += e[2].elapsed_time(e[3])
+    dev_ms = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
+    ms = max_over_ranks(dist, dev_ms)
+    stage_ms = {kk: vv / args.steps for kk, vv in stage.items()}
+
+    # Flat single-level selector on the same inputs (its own launches).
+    fe0, fe1 = events(2)
+    api.select_flat(q, p.pyr, C=w.C, K=w.K, causal=w.causal, H_kv=w.H_kv)
+    fe0.record(stream)
+    for _ in range(args.steps):
+        api.select_flat(q, p.pyr, C=w.C, K=w.K, causal=w.causal, H_kv=w.H_kv, out=p.sel)
+    fe1.record(stream)
+    torch.cuda.synchronize()
+    flat_ms = fe0.elapsed_time(fe1) / args.steps
+
+    # End to end through the public API from pinned host buffers.
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = torch.empty(p.out.shape, dtype=p.out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    e2e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    ee0, ee1 = events(2)
+    ee0.record(stream)
+    for _ in range(e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        p(dq, dk, dv)
+        hout.copy_(p.out, non_blocking=True)
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(dist, ee0.elapsed_time(ee1) / e2e_steps)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = hout.numel() * hout.element_size()
+    del hq, hk, hv, hout, dq, dk, dv
+
+    decode = None
+    if not args.no_decode:
+        del x
+        torch.cuda.empty_cache()
+        decode = time_decode(workloads.DECODE[args.decode_workload])
+
+    pk, pk_kind = peaks()
+    # Roofline of the dominant stage (the attention kernel: one launch per step).
+    a_bytes = attn_bytes(w)
+    a_ms = stage_ms["attn"]
+    roof = {"kernel": "sparse_attn_fwd", "bound": "hbm", "achieved": a_bytes / (a_ms * 1e-3) / 1e9,
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_kind": pk_kind, "traffic": None,
+            "algorithmic_bytes": a_bytes}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+
+    tokens = w.B * w.N * world
+    line = {
+        "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "C": w.C,
+                   "g": 2, "K": w.K, "q_tile": 4, "causal": w.causal, "structure": w.structure,
+                   "l2": "inputs larger than L2 (q alone is %.0f MB)" % (q.numel() * q.element_size() / 1e6)},
+        "stages_ms": stage_ms, "flat_select_ms": flat_ms,
+        "select_speedup_vs_flat": flat_ms / stage_ms["select"] if stage_ms["select"] > 0 else None,
+        "decode": decode,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches, "roofline": roof, "clocks": clk.summary(), "wall_s": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        xh = workloads.prefill_inputs(w, device=dev)
+        line["cpu_baseline"] = cpu_baseline(w, xh, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line))
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="needle_256k", choices=sorted(workloads.PREFILL))
+    ap.add_argument("--decode-workload", default="decode_64x128k", choices=sorted(workloads.DECODE))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

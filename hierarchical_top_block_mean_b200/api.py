@@ -1,0 +1,252 @@
+"""Public Python API over the C ABI (include/pisa.h).
+
+PyTorch supplies device memory and streams; every computation runs in the
+library's CUDA kernels. Tensors must be contiguous CUDA tensors in bfloat16
+or float32 ([B, H, N, d] for q/k/v); results are written into the given (or
+newly allocated) output tensors on the current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float32: _lib.DTYPE_F32, torch.bfloat16: _lib.DTYPE_BF16}
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(_lib.lib().pisa_launch_count())
+
+
+def pyramid_geometry(N: int, C: int, g: int = 2):
+    """(L, offsets): level l (1..L) occupies rows offsets[l-1]:offsets[l]."""
+    L = ctypes.c_int32()
+    _lib.call("pisa_pyramid_geometry", N, C, g, ctypes.byref(L), None)
+    offs = (ctypes.c_int64 * (L.value + 1))()
+    _lib.call("pisa_pyramid_geometry", N, C, g, ctypes.byref(L), offs)
+    return L.value, list(offs)
+
+
+def pyramid_rows(N: int, C: int) -> int:
+    return int(_lib.lib().pisa_pyramid_rows(N, C))
+
+
+@dataclass(frozen=True)
+class Problem:
+    """Prefill shape and hyper-parameters (paper: C leaf size, g = 2, K, Q_tile = 4)."""
+    B: int
+    N: int
+    H_q: int
+    H_kv: int
+    d: int
+    C: int
+    K: int
+    causal: bool
+    dtype: torch.dtype
+    scale: float = 0.0
+    g: int = 2
+    q_tile: int = 4
+
+    @staticmethod
+    def of(q: torch.Tensor, k: torch.Tensor, *, C: int, K: int, causal: bool, scale: float = 0.0) -> "Problem":
+        B, H_q, N, d = q.shape
+        Bk, H_kv, Nk, dk = k.shape
+        if (B, N, d) != (Bk, Nk, dk):
+            raise ValueError(f"q {tuple(q.shape)} and k {tuple(k.shape)} disagree")
+        if q.dtype != k.dtype or q.dtype not in _DT:
+            raise ValueError("q and k must share dtype float32 or bfloat16")
+        return Problem(B, N, H_q, H_kv, d, C, K, bool(causal), q.dtype, scale)
+
+    def cstruct(self) -> _lib.Config:
+        return _lib.Config(self.B, self.N, self.H_q, self.H_kv, self.d, self.C, self.g, self.K, self.q_tile,
+                           int(self.causal), _DT[self.dtype], self.scale)
+
+    @property
+    def R(self) -> int:
+        return pyramid_rows(self.N, self.C)
+
+    def workspace_bytes(self) -> int:
+        return int(_lib.lib().pisa_select_workspace_bytes(ctypes.byref(self.cstruct())))
+
+
+def build_pyramid(k: torch.Tensor, *, C: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Mean-pooled key pyramid of k [B, H_kv, N, d] -> fp32 [B, H_kv, R, d]."""
+    _need(k, "k")
+    B, H, N, d = k.shape
+    pr = Problem(B, N, H, H, d, C, 1, False, k.dtype)
+    if out is None:
+        out = torch.empty((B, H, pr.R, d), dtype=torch.float32, device=k.device)
+    _need(out, "out", torch.float32)
+    _lib.call("pisa_build_pyramid", ctypes.byref(pr.cstruct()), _p(k), _p(out), _stream(k))
+    return out
+
+
+def select(q, k, pyr, *, C: int, K: int, causal: bool, scale: float = 0.0, out=None, score=None,
+           workspace=None):
+    """PISA coarse-to-fine top-K leaf blocks: sel [B, H_kv, N, K] int32 (ascending, -1 padded)."""
+    for t, n in ((q, "q"), (k, "k"), (pyr, "pyr")):
+        _need(t, n)
+    pr = Problem.of(q, k, C=C, K=K, causal=causal, scale=scale)
+    if out is None:
+        out = torch.empty((pr.B, pr.H_kv, pr.N, K), dtype=torch.int32, device=q.device)
+    need = pr.workspace_bytes()
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _lib.call("pisa_select", ctypes.byref(pr.cstruct()), _p(q), _p(k), _p(pyr), _p(out), _p(score), _p(workspace),
+              workspace.numel() * workspace.element_size(), _stream(q))
+    return out
+
+
+def select_flat(q, pyr, *, C: int, K: int, causal: bool, H_kv: int, scale: float = 0.0, out=None):
+    """Flat single-level top-K over all leaf summaries: sel [B, H_kv, N, K] int32."""
+    _need(q, "q")
+    _need(pyr, "pyr", torch.float32)
+    B, H_q, N, d = q.shape
+    pr = Problem(B, N, H_q, H_kv, d, C, K, bool(causal), q.dtype, scale)
+    if out is None:
+        out = torch.empty((B, H_kv, N, K), dtype=torch.int32, device=q.device)
+    _lib.call("pisa_select_flat", ctypes.byref(pr.cstruct()), _p(q), _p(pyr), _p(out), _stream(q))
+    return out
+
+
+def sparse_attn_fwd(q, k, v, sel, *, C: int, causal: bool, scale: float = 0.0, out=None, lse=None,
+                    want_lse: bool = True):
+    """Block-sparse attention over the selected leaf blocks: (out [B,H_q,N,d], lse [B,H_q,N] or None)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    _need(sel, "sel", torch.int32)
+    K = sel.shape[-1]
+    pr = Problem.of(q, k, C=C, K=K, causal=causal, scale=scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    _lib.call("pisa_sparse_attn_fwd", ctypes.byref(pr.cstruct()), _p(q), _p(k), _p(v), _p(sel), _p(out), _p(lse),
+              _stream(q))
+    return out, lse
+
+
+class Prefill:
+    """Reusable prefill pipeline for one problem shape: pyramid, PISA select
+    and block-sparse attention, with all buffers allocated once."""
+
+    def __init__(self, pr: Problem, device="cuda"):
+        self.pr = pr
+        dev = torch.device(device)
+        self.cfg = pr.cstruct()
+        self.pyr = torch.empty((pr.B, pr.H_kv, pr.R, pr.d), dtype=torch.float32, device=dev)
+        self.sel = torch.empty((pr.B, pr.H_kv, pr.N, pr.K), dtype=torch.int32, device=dev)
+        self.ws = torch.empty(max(pr.workspace_bytes(), 16), dtype=torch.uint8, device=dev)
+        self.out = torch.empty((pr.B, pr.H_q, pr.N, pr.d), dtype=pr.dtype, device=dev)
+        self.lse = torch.empty((pr.B, pr.H_q, pr.N), dtype=torch.float32, device=dev)
+
+    def pyramid(self, k):
+        _lib.call("pisa_build_pyramid", ctypes.byref(self.cfg), _p(k), _p(self.pyr), _stream(k))
+
+    def select(self, q, k):
+        _lib.call("pisa_select", ctypes.byref(self.cfg), _p(q), _p(k), _p(self.pyr), _p(self.sel), None,
+                  _p(self.ws), self.ws.numel(), _stream(q))
+
+    def attend(self, q, k, v):
+        _lib.call("pisa_sparse_attn_fwd", ctypes.byref(self.cfg), _p(q), _p(k), _p(v), _p(self.sel), _p(self.out),
+                  _p(self.lse), _stream(q))
+
+    def __call__(self, q, k, v):
+        self.pyramid(k)
+        self.select(q, k)
+        self.attend(q, k, v)
+        return self.out
+
+
+def prefill(q, k, v, *, C: int, K: int, causal: bool, scale: float = 0.0):
+    """Pyramid + PISA selection + block-sparse attention in one call: (out, lse, sel)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    p = Prefill(Problem.of(q, k, C=C, K=K, causal=causal, scale=scale), q.device)
+    p(q, k, v)
+    return p.out, p.lse, p.sel
+
+
+class DecodeState:
+    """Caller-side decode state for S sequences of capacity cap: KV caches,
+    the cached mean pyramid, per-sequence lengths and a device status word."""
+
+    def __init__(self, *, S: int, cap: int, H_q: int, H_kv: int, d: int, C: int, K: int,
+                 dtype=torch.bfloat16, scale: float = 0.0, device="cuda", k_cache=None, v_cache=None, lens=None):
+        dev = torch.device(device)
+        self.cfg = _lib.DecodeConfig(S, cap, H_q, H_kv, d, C, 2, K, _DT[dtype], scale)
+        self.S, self.cap, self.H_q, self.H_kv, self.d, self.C, self.K = S, cap, H_q, H_kv, d, C, K
+        self.dtype = dtype
+        R = int(_lib.lib().pisa_decode_pyramid_rows(ctypes.byref(self.cfg)))
+        if R <= 0:
+            raise _lib.PisaError("pisa_decode_pyramid_rows", 1)
+        self.R = R
+        self.k_cache = k_cache if k_cache is not None else torch.zeros((S, H_kv, cap, d), dtype=dtype, device=dev)
+        self.v_cache = v_cache if v_cache is not None else torch.zeros((S, H_kv, cap, d), dtype=dtype, device=dev)
+        self.len = lens if lens is not None else torch.zeros(S, dtype=torch.int32, device=dev)
+        for t, n in ((self.k_cache, "k_cache"), (self.v_cache, "v_cache")):
+            _need(t, n, dtype)
+        _need(self.len, "len", torch.int32)
+        self.pyr = torch.zeros((S, H_kv, R, d), dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.sel = torch.empty((S, H_kv, K), dtype=torch.int32, device=dev)
+        self.out = torch.empty((S, H_q, d), dtype=dtype, device=dev)
+        self.lse = torch.empty((S, H_q), dtype=torch.float32, device=dev)
+
+    def init(self):
+        """Builds each sequence's pyramid over its first len[s] cached tokens."""
+        _lib.call("pisa_decode_init", ctypes.byref(self.cfg), _p(self.k_cache), _p(self.pyr), _p(self.len),
+                  _stream(self.pyr))
+
+    def append(self, k_new, v_new):
+        _lib.call("pisa_decode_append", ctypes.byref(self.cfg), _p(k_new), _p(v_new), _p(self.k_cache),
+                  _p(self.v_cache), _p(self.pyr), _p(self.len), _p(self.status), _stream(self.pyr))
+
+    def select(self, q_new):
+        _lib.call("pisa_decode_select", ctypes.byref(self.cfg), _p(q_new), _p(self.k_cache), _p(self.pyr),
+                  _p(self.len), _p(self.sel), _stream(self.pyr))
+        return self.sel
+
+    def attend(self, q_new, sel=None):
+        s = self.sel if sel is None else sel
+        _lib.call("pisa_decode_attn", ctypes.byref(self.cfg), _p(q_new), _p(self.k_cache), _p(self.v_cache),
+                  _p(self.len), _p(s), _p(self.out), _p(self.lse), _stream(self.pyr))
+        return self.out
+
+    def step(self, q_new, k_new, v_new, keep_sel: bool = True):
+        """Append + select + attend for every sequence."""
+        _lib.call("pisa_decode_step", ctypes.byref(self.cfg), _p(q_new), _p(k_new), _p(v_new), _p(self.k_cache),
+                  _p(self.v_cache), _p(self.pyr), _p(self.len), _p(self.sel) if keep_sel else None, _p(self.out),
+                  _p(self.lse), _p(self.status), _stream(self.pyr))
+        return self.out
+
+    def level_offsets(self):
+        return pyramid_geometry(self.cap, self.C)[1]
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,219 @@
+// C ABI entry points (include/pisa.h): host-side validation, layout
+// arithmetic and dispatch to the kernels. Nothing here allocates device
+// memory, synchronises or keeps state besides the launch counter.
+#include <atomic>
+#include <cmath>
+
+#include "kernels.cuh"
+#include "pyramid.cuh"
+#include "select2.cuh"
+
+namespace pisa {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline pisa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PISA_OK : PISA_ERR_CUDA; }
+
+pisa_status check_shape(int H_q, int H_kv, int d, int C, int g, int K, int dtype) {
+  if (H_q < 1 || H_kv < 1 || d < 1 || C < 1 || K < 1) return PISA_ERR_INVALID_ARGUMENT;
+  if (H_q % H_kv != 0) return PISA_ERR_INVALID_ARGUMENT;
+  if (dtype != PISA_DTYPE_F32 && dtype != PISA_DTYPE_BF16) return PISA_ERR_INVALID_ARGUMENT;
+  const int G = H_q / H_kv;
+  if (g != 2 || (C != 32 && C != 64) || (d != 64 && d != 128) || K > kMaxK) return PISA_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PISA_ERR_UNSUPPORTED;
+  return PISA_OK;
+}
+
+pisa_status check_cfg(const pisa_config* c) {
+  if (!c) return PISA_ERR_INVALID_ARGUMENT;
+  if (c->B < 1 || c->N < 1 || (c->causal != 0 && c->causal != 1)) return PISA_ERR_INVALID_ARGUMENT;
+  pisa_status s = check_shape(c->H_q, c->H_kv, c->d, c->C, c->g, c->K, c->dtype);
+  if (s != PISA_OK) return s;
+  if (c->q_tile != 4) return PISA_ERR_UNSUPPORTED;
+  return PISA_OK;
+}
+
+pisa_status check_dcfg(const pisa_decode_config* c) {
+  if (!c) return PISA_ERR_INVALID_ARGUMENT;
+  if (c->S < 1 || c->cap < 1) return PISA_ERR_INVALID_ARGUMENT;
+  return check_shape(c->H_q, c->H_kv, c->d, c->C, c->g, c->K, c->dtype);
+}
+
+PrefillArgs args_of(const pisa_config* c) {
+  PrefillArgs a{c->B, c->N, c->H_q, c->H_kv, c->d, c->C, c->K, c->causal, c->dtype, c->scale};
+  if (!(a.scale > 0.f)) a.scale = 1.0f / std::sqrt(static_cast<float>(c->d));
+  return a;
+}
+
+DecodeArgs dargs_of(const pisa_decode_config* c) {
+  DecodeArgs a{c->S, c->cap, c->H_q, c->H_kv, c->d, c->C, c->K, c->dtype, c->scale};
+  if (!(a.scale > 0.f)) a.scale = 1.0f / std::sqrt(static_cast<float>(c->d));
+  return a;
+}
+
+}  // namespace
+}  // namespace pisa
+
+using namespace pisa;
+
+extern "C" {
+
+const char* pisa_status_string(int32_t status) {
+  switch (status) {
+    case PISA_OK: return "PISA_OK";
+    case PISA_ERR_INVALID_ARGUMENT: return "PISA_ERR_INVALID_ARGUMENT";
+    case PISA_ERR_UNSUPPORTED: return "PISA_ERR_UNSUPPORTED";
+    case PISA_ERR_WORKSPACE: return "PISA_ERR_WORKSPACE";
+    case PISA_ERR_CAPACITY: return "PISA_ERR_CAPACITY";
+    case PISA_ERR_CUDA: return "PISA_ERR_CUDA";
+    case PISA_ERR_DEVICE: return "PISA_ERR_DEVICE";
+    default: return "PISA_ERR_UNKNOWN";
+  }
+}
+
+int32_t pisa_version(void) { return 100; }
+
+uint64_t pisa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+pisa_status pisa_pyramid_geometry(int64_t N, int32_t C, int32_t g, int32_t* num_levels_out, int64_t* level_offsets) {
+  if (N < 1 || C < 1 || g != 2 || !num_levels_out) return PISA_ERR_INVALID_ARGUMENT;
+  const int L = num_levels(N, C);
+  *num_levels_out = L;
+  if (level_offsets) {
+    int64_t acc = 0;
+    for (int l = 1; l <= L; ++l) {
+      level_offsets[l - 1] = acc;
+      acc += level_size(N, C, l);
+    }
+    level_offsets[L] = acc;
+  }
+  return PISA_OK;
+}
+
+int64_t pisa_pyramid_rows(int64_t N, int32_t C) {
+  if (N < 1 || C < 1) return 0;
+  return make_layout(N, C).R;
+}
+
+pisa_status pisa_build_pyramid(const pisa_config* cfg, const void* k, float* pyr, void* stream) {
+  pisa_status s = check_cfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!k || !pyr || !aligned16(k) || !aligned16(pyr)) return PISA_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(cfg->N, cfg->C);
+  return from_cuda(launch_build_pyramid(cfg->dtype, cfg->d, k, pyr, lay, cfg->N, cfg->N, nullptr,
+                                        cfg->B * cfg->H_kv, cfg->H_kv, cfg->N, cfg->C, as_stream(stream)));
+}
+
+size_t pisa_select_workspace_bytes(const pisa_config* cfg) {
+  if (check_cfg(cfg) != PISA_OK) return 0;
+  if (cfg->dtype != PISA_DTYPE_BF16) return 0;  // the fp32 path selects row by row without scratch
+  return select2_workspace_bytes(args_of(cfg));
+}
+
+pisa_status pisa_select(const pisa_config* cfg, const void* q, const void* k, const float* pyr, int32_t* sel,
+                        float* sel_score, void* ws, size_t ws_bytes, void* stream) {
+  pisa_status s = check_cfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!q || !k || !pyr || !sel || !aligned16(q) || !aligned16(k) || !aligned16(pyr) || !aligned16(sel))
+    return PISA_ERR_INVALID_ARGUMENT;
+  const PrefillArgs a = args_of(cfg);
+  const Layout lay = make_layout(cfg->N, cfg->C);
+  if (cfg->dtype == PISA_DTYPE_BF16) {
+    const size_t need = select2_workspace_bytes(a);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return PISA_ERR_WORKSPACE;
+    return from_cuda(launch_select2(a, q, k, pyr, lay, sel, sel_score, ws, as_stream(stream)));
+  }
+  return from_cuda(launch_select_rows(a, q, k, pyr, lay, sel, sel_score, as_stream(stream)));
+}
+
+pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float* pyr, int32_t* sel, void* stream) {
+  pisa_status s = check_cfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!q || !pyr || !sel || !aligned16(q) || !aligned16(pyr) || !aligned16(sel)) return PISA_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(cfg->N, cfg->C);
+  return from_cuda(launch_flat_rows(args_of(cfg), q, pyr, lay.R, sel, as_stream(stream)));
+}
+
+pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
+                                 const int32_t* sel, void* out, float* lse, void* stream) {
+  pisa_status s = check_cfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!q || !k || !v || !sel || !out) return PISA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return PISA_ERR_INVALID_ARGUMENT;
+  return from_cuda(launch_attn_rows(args_of(cfg), q, k, v, sel, out, lse, as_stream(stream)));
+}
+
+int64_t pisa_decode_pyramid_rows(const pisa_decode_config* cfg) {
+  if (check_dcfg(cfg) != PISA_OK) return 0;
+  return make_layout(cfg->cap, cfg->C).R;
+}
+
+pisa_status pisa_decode_init(const pisa_decode_config* cfg, const void* k_cache, float* pyr, const int32_t* len,
+                             void* stream) {
+  pisa_status s = check_dcfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!k_cache || !pyr || !len || !aligned16(k_cache) || !aligned16(pyr)) return PISA_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(cfg->cap, cfg->C);
+  return from_cuda(launch_build_pyramid(cfg->dtype, cfg->d, k_cache, pyr, lay, cfg->cap, 0, len,
+                                        cfg->S * cfg->H_kv, cfg->H_kv, cfg->cap, cfg->C, as_stream(stream)));
+}
+
+pisa_status pisa_decode_append(const pisa_decode_config* cfg, const void* k_new, const void* v_new, void* k_cache,
+                               void* v_cache, float* pyr, int32_t* len, int32_t* status, void* stream) {
+  pisa_status s = check_dcfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!k_new || !v_new || !k_cache || !v_cache || !pyr || !len || !status) return PISA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(pyr)) return PISA_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(cfg->cap, cfg->C);
+  return from_cuda(launch_decode_append(dargs_of(cfg), lay, k_new, v_new, k_cache, v_cache, pyr, len, status,
+                                        as_stream(stream)));
+}
+
+pisa_status pisa_decode_select(const pisa_decode_config* cfg, const void* q_new, const void* k_cache,
+                               const float* pyr, const int32_t* len, int32_t* sel, void* stream) {
+  pisa_status s = check_dcfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!q_new || !k_cache || !pyr || !len || !sel) return PISA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q_new) || !aligned16(k_cache) || !aligned16(pyr)) return PISA_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(cfg->cap, cfg->C);
+  return from_cuda(launch_decode_rows(dargs_of(cfg), lay, 1, q_new, k_cache, nullptr, pyr, len, sel, nullptr,
+                                      nullptr, as_stream(stream)));
+}
+
+pisa_status pisa_decode_attn(const pisa_decode_config* cfg, const void* q_new, const void* k_cache,
+                             const void* v_cache, const int32_t* len, const int32_t* sel, void* out, float* lse,
+                             void* stream) {
+  pisa_status s = check_dcfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!q_new || !k_cache || !v_cache || !len || !sel || !out) return PISA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q_new) || !aligned16(k_cache) || !aligned16(v_cache)) return PISA_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(cfg->cap, cfg->C);
+  return from_cuda(launch_decode_rows(dargs_of(cfg), lay, 2, q_new, k_cache, v_cache, nullptr, len,
+                                      const_cast<int32_t*>(sel), out, lse, as_stream(stream)));
+}
+
+pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, const void* k_new, const void* v_new,
+                             void* k_cache, void* v_cache, float* pyr, int32_t* len, int32_t* sel, void* out,
+                             float* lse, int32_t* status, void* stream) {
+  pisa_status s = check_dcfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!q_new || !k_new || !v_new || !k_cache || !v_cache || !pyr || !len || !out || !status)
+    return PISA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q_new) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(pyr))
+    return PISA_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(cfg->cap, cfg->C);
+  const DecodeArgs a = dargs_of(cfg);
+  cudaError_t e = launch_decode_append(a, lay, k_new, v_new, k_cache, v_cache, pyr, len, status, as_stream(stream));
+  if (e != cudaSuccess) return PISA_ERR_CUDA;
+  return from_cuda(
+      launch_decode_rows(a, lay, 3, q_new, k_cache, v_cache, pyr, len, sel, out, lse, as_stream(stream)));
+}
+
+}  // extern "C"

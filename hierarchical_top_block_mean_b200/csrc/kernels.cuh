@@ -1,0 +1,39 @@
+// Launchers behind the C ABI. Every launcher enqueues on `st`, counts its
+// launches and returns the launch status; none synchronises or allocates.
+#pragma once
+
+#include "common.cuh"
+
+namespace pisa {
+
+// Prefill problem with the scale resolved (kernel parameter, passed by value).
+struct PrefillArgs {
+  int B, N, H_q, H_kv, d, C, K, causal, dtype;
+  float scale;
+};
+
+// Decode problem with the scale resolved.
+struct DecodeArgs {
+  int S, cap, H_q, H_kv, d, C, K, dtype;
+  float scale;
+};
+
+// ---- warp-per-row kernels (fp32 path)
+cudaError_t launch_select_rows(const PrefillArgs& a, const void* q, const void* k, const float* pyr,
+                               const Layout& lay, int32_t* sel, float* sel_score, cudaStream_t st);
+cudaError_t launch_attn_rows(const PrefillArgs& a, const void* q, const void* k, const void* v, const int32_t* sel,
+                             void* out, float* lse, cudaStream_t st);
+cudaError_t launch_flat_rows(const PrefillArgs& a, const void* q, const float* pyr, int64_t R, int32_t* sel,
+                             cudaStream_t st);
+
+// ---- decode
+cudaError_t launch_decode_append(const DecodeArgs& a, const Layout& lay, const void* k_new, const void* v_new,
+                                 void* k_cache, void* v_cache, float* pyr, int32_t* len, int32_t* status,
+                                 cudaStream_t st);
+// mode bit 1: select (writes sel if not null), bit 2: attend (reads sel from
+// memory when bit 1 is clear).
+cudaError_t launch_decode_rows(const DecodeArgs& a, const Layout& lay, int mode, const void* q_new,
+                               const void* k_cache, const void* v_cache, const float* pyr, const int32_t* len,
+                               int32_t* sel, void* out, float* lse, cudaStream_t st);
+
+}  // namespace pisa

@@ -1,0 +1,195 @@
+/*
+ * pisa.h — C ABI of the B200 (sm_100a) PISA hot path: mean-pooled key
+ * pyramid, coarse-to-fine top-K block selection, flat single-level block
+ * selection, block-sparse attention forward, and the decode step.
+ *
+ * The method is "Block Sparse Attention with Log-Linear Complexity"
+ * (Tang, Qin, Pan, Li, Liu). Citations below name sections of its hyper.ai
+ * page (the translated paper body): §BSA "Block-sparse attention",
+ * §Pyramid "Pyramid key-block hierarchy", §TopK "Coarse-to-fine Top-K
+ * selection", §Kernels "Kernel implementation", §Complexity.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named q, k, v, pyr, sel, out, lse, ws, k_cache, v_cache, len,
+ *     status are DEVICE pointers to memory the caller owns. The library never
+ *     allocates, never synchronises the device and keeps no state between
+ *     calls (except the launch counter of pisa_launch_count).
+ *   - Tensors are dense and row-major: q [B, H_q, N, d]; k, v [B, H_kv, N, d];
+ *     query head h' belongs to kv head h' / G_Q with G_Q = H_q / H_kv.
+ *   - dtype selects the storage of q, k, v and out: PISA_DTYPE_BF16 or
+ *     PISA_DTYPE_F32. Pyramids are always fp32; lse is always fp32.
+ *   - Blocks, levels and indices are 0-based (the paper's root block "1" is
+ *     block 0 here). Level 1 holds the leaf blocks of C keys; level l >= 2
+ *     merges pairs (g = 2) of level l-1.
+ *   - Causal reading (the paper does not state one): a block is usable by
+ *     the query at position t iff its first key is <= t; leaf scores and
+ *     attention use only keys <= t.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All work is enqueued on it; results are ready when the stream is.
+ *   - Arguments are validated on the host before anything is enqueued. A
+ *     rejected call returns its error and enqueues nothing. A launch failure
+ *     returns PISA_ERR_CUDA. Nothing in the library traps or waits without a
+ *     bound.
+ *   - Supported shapes: g = 2; C in {32, 64}; d in {64, 128}; 1 <= K <= 16;
+ *     q_tile = 4; G_Q in {1, 2, 4, 8}; other values return
+ *     PISA_ERR_UNSUPPORTED.
+ */
+#ifndef PISA_H_
+#define PISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PISA_OK = 0,
+  PISA_ERR_INVALID_ARGUMENT = 1, /* null pointer, non-positive size, H_q % H_kv != 0, ... */
+  PISA_ERR_UNSUPPORTED = 2,      /* valid but outside the supported shapes listed above   */
+  PISA_ERR_WORKSPACE = 3,        /* ws is null or smaller than pisa_select_workspace_bytes */
+  PISA_ERR_CAPACITY = 4,         /* decode: a sequence is full (written to the status word) */
+  PISA_ERR_CUDA = 5,             /* a CUDA launch or runtime call failed                   */
+  PISA_ERR_DEVICE = 6            /* a device-side check failed (written to a status word)  */
+} pisa_status;
+
+typedef enum { PISA_DTYPE_F32 = 0, PISA_DTYPE_BF16 = 1 } pisa_dtype;
+
+/* Prefill problem. scale <= 0 selects 1/sqrt(d) (§BSA). causal is 0 or 1. */
+typedef struct {
+  int32_t B, N, H_q, H_kv, d, C, g, K, q_tile, causal;
+  int32_t dtype; /* pisa_dtype */
+  float scale;
+} pisa_config;
+
+/* Decode problem: S independent sequences, each with room for cap tokens. */
+typedef struct {
+  int32_t S, cap, H_q, H_kv, d, C, g, K;
+  int32_t dtype; /* pisa_dtype */
+  float scale;
+} pisa_decode_config;
+
+/* Human-readable name of a status code (static storage). */
+const char* pisa_status_string(int32_t status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int32_t pisa_version(void);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all entry points). Host-side counter; for accounting and tests. */
+uint64_t pisa_launch_count(void);
+
+/*
+ * Pyramid geometry (host only, pure integer arithmetic) — §Pyramid level
+ * sizes: M_0 = N, M_1 = ceil(N / C), M_{l+1} = ceil(M_l / g) until M_L = 1.
+ * Writes L to *num_levels. If level_offsets is not NULL it receives L + 1
+ * entries: level l (1..L) occupies rows [level_offsets[l-1], level_offsets[l])
+ * of a head's pyramid, finest level first, and level_offsets[L] is the row
+ * count R. Returns PISA_ERR_INVALID_ARGUMENT for N < 1, C < 1 or g != 2.
+ */
+pisa_status pisa_pyramid_geometry(int64_t N, int32_t C, int32_t g, int32_t* num_levels, int64_t* level_offsets);
+
+/* Rows R of one head's pyramid for N tokens (0 on invalid input). */
+int64_t pisa_pyramid_rows(int64_t N, int32_t C);
+
+/*
+ * Mean-pooled key pyramid — §Pyramid summary recursion: a leaf summary is the
+ * mean of its (up to C) raw keys, every higher summary the unweighted mean of
+ * the children the block has.
+ *   k   : [B, H_kv, N, d] in cfg->dtype.
+ *   pyr : [B, H_kv, R, d] fp32, R = pisa_pyramid_rows(N, C), laid out as in
+ *         pisa_pyramid_geometry. Fully overwritten.
+ */
+pisa_status pisa_build_pyramid(const pisa_config* cfg, const void* k, float* pyr, void* stream);
+
+/* Bytes of scratch workspace pisa_select needs for cfg (0 on invalid cfg). */
+size_t pisa_select_workspace_bytes(const pisa_config* cfg);
+
+/*
+ * Coarse-to-fine top-K leaf-block selection — §TopK (candidate sets, keep-all
+ * rule, LSE block score) with the GQA score sum and the two-stage split of
+ * §Kernels: stage 1 routes levels L..2, stage 2 groups queries by candidate
+ * leaf into tiles of q_tile queries, scores leaves by their exact raw-key LSE
+ * and keeps the final top K. Ties go to the lower block index.
+ *   q        : [B, H_q, N, d];  k : [B, H_kv, N, d];  pyr : from pisa_build_pyramid.
+ *   sel      : [B, H_kv, N, K] int32 — selected leaf blocks per (kv head, query),
+ *              ascending, padded with -1 when fewer than K blocks are valid.
+ *   sel_score: NULL, or [B, H_kv, N, K] fp32 — the leaf-level score of each
+ *              selected block (NaN when the leaf level was kept unscored, or
+ *              for padding).
+ *   ws       : device scratch of at least pisa_select_workspace_bytes(cfg)
+ *              bytes, caller-owned, contents on entry ignored.
+ */
+pisa_status pisa_select(const pisa_config* cfg, const void* q, const void* k, const float* pyr, int32_t* sel,
+                        float* sel_score, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Flat single-level selection — §BSA: a flat method scores all M = ceil(N/C)
+ * leaf summaries per query. Score reading: u_i = sum over the group of
+ * scale * q_{h',t} . kbar^{(1)}_i; top K with the same validity, tie, order
+ * and padding rules as pisa_select. Needs no workspace.
+ *   q : [B, H_q, N, d];  pyr : [B, H_kv, R, d] (only level 1 is read);
+ *   sel : [B, H_kv, N, K] int32.
+ */
+pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float* pyr, int32_t* sel, void* stream);
+
+/*
+ * Block-sparse attention forward — §BSA:
+ *   o_t = sum_{j in T_t} exp(scale q_t.k_j) v_j / sum_{j in T_t} exp(scale q_t.k_j)
+ * over the raw keys of the selected leaf blocks T_t (shared by the query heads
+ * of a GQA group; keys > t excluded when causal). Negative sel entries are
+ * padding; every row must select at least one usable block.
+ *   sel : [B, H_kv, N, K] int32;  out : [B, H_q, N, d] in cfg->dtype;
+ *   lse : NULL or [B, H_q, N] fp32, natural-log softmax denominator.
+ */
+pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
+                                 const int32_t* sel, void* out, float* lse, void* stream);
+
+/* ---------------------------------------------------------------- decode
+ * §Kernels, decoding: the mean pyramid is cached; per new token only the
+ * current leaf mean and its ancestor path are updated, and one fused kernel
+ * selects from the coarsest level down to the leaves, scoring raw key blocks
+ * directly.
+ *   k_cache, v_cache : [S, H_kv, cap, d] in dtype.
+ *   pyr              : [S, H_kv, R_cap, d] fp32, R_cap = pisa_decode_pyramid_rows;
+ *                      level l of every sequence sits at the offset it has for
+ *                      cap tokens (pisa_pyramid_geometry(cap, ...)).
+ *   len              : [S] int32 device, tokens held per sequence.
+ *   status           : one int32 device word; kernels store PISA_ERR_CAPACITY
+ *                      there when a sequence is full (that sequence is skipped)
+ *                      and never clear it.
+ */
+int64_t pisa_decode_pyramid_rows(const pisa_decode_config* cfg);
+
+/* Builds every sequence's pyramid over its first len[s] cached keys. */
+pisa_status pisa_decode_init(const pisa_decode_config* cfg, const void* k_cache, float* pyr, const int32_t* len,
+                             void* stream);
+
+/* Appends k_new/v_new [S, H_kv, d] at position len[s], updates that leaf
+ * mean and its ancestors, then increments len[s]. */
+pisa_status pisa_decode_append(const pisa_decode_config* cfg, const void* k_new, const void* v_new, void* k_cache,
+                               void* v_cache, float* pyr, int32_t* len, int32_t* status, void* stream);
+
+/* Selects K leaf blocks for q_new [S, H_q, d], the query at position
+ * len[s] - 1 (every block of the sequence is valid). sel: [S, H_kv, K]. */
+pisa_status pisa_decode_select(const pisa_decode_config* cfg, const void* q_new, const void* k_cache,
+                               const float* pyr, const int32_t* len, int32_t* sel, void* stream);
+
+/* Attention of q_new over the selected blocks of each sequence's first
+ * len[s] tokens. out: [S, H_q, d] in dtype; lse: NULL or [S, H_q] fp32. */
+pisa_status pisa_decode_attn(const pisa_decode_config* cfg, const void* q_new, const void* k_cache,
+                             const void* v_cache, const int32_t* len, const int32_t* sel, void* out, float* lse,
+                             void* stream);
+
+/* One decode step in one launch: append, select and attend for every
+ * sequence. sel may be NULL (selection kept on chip); otherwise [S, H_kv, K]. */
+pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, const void* k_new, const void* v_new,
+                             void* k_cache, void* v_cache, float* pyr, int32_t* len, int32_t* sel, void* out,
+                             float* lse, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PISA_H_ */

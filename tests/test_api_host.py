@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/pisa.h declares, its integer pyramid geometry matches
+the oracle bit for bit, and argument validation rejects bad calls before
+anything is enqueued."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from hierarchical_top_block_mean_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "pisa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(pisa_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.lib()
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_status_strings_and_version():
+    lib = _lib.lib()
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.pisa_status_string(code).decode() == name
+    assert lib.pisa_version() >= 100
+
+
+@pytest.mark.parametrize("N,C", [(1, 32), (5, 32), (1024, 32), (1000, 64), (16384, 64), (131328, 64),
+                                 (262144, 64), (77777, 32)])
+def test_geometry_matches_oracle(oracle, N, C):
+    from hierarchical_top_block_mean_b200 import pyramid_geometry, pyramid_rows
+    L, offs = pyramid_geometry(N, C)
+    sizes, ooffs = oracle.geometry(N, C)
+    assert L == len(sizes) - 1
+    assert offs == list(ooffs)
+    assert pyramid_rows(N, C) == ooffs[-1]
+
+
+def _cfg(**kw):
+    base = dict(B=1, N=256, H_q=4, H_kv=1, d=64, C=32, g=2, K=4, q_tile=4, causal=1, dtype=1, scale=0.0)
+    base.update(kw)
+    return _lib.Config(*[base[f] for f, _ in _lib.Config._fields_])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=0), 1), (dict(B=0), 1), (dict(H_q=6, H_kv=4), 1), (dict(dtype=7), 1), (dict(causal=2), 1),
+    (dict(g=3), 2), (dict(C=16), 2), (dict(d=96), 2), (dict(K=17), 2), (dict(q_tile=8), 2),
+    (dict(H_q=12, H_kv=1), 2),
+])
+def test_invalid_configs_rejected_before_launch(kw, code):
+    lib = _lib.lib()
+    before = lib.pisa_launch_count()
+    dummy = ctypes.c_void_p(256)
+    cfg = _cfg(**kw)
+    assert lib.pisa_build_pyramid(ctypes.byref(cfg), dummy, dummy, None) == code
+    assert lib.pisa_select(ctypes.byref(cfg), dummy, dummy, dummy, dummy, None, dummy, 1 << 30, None) == code
+    assert lib.pisa_select_flat(ctypes.byref(cfg), dummy, dummy, dummy, None) == code
+    assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), dummy, dummy, dummy, dummy, dummy, None, None) == code
+    assert lib.pisa_select_workspace_bytes(ctypes.byref(cfg)) == 0
+    assert lib.pisa_launch_count() == before
+
+
+def test_null_and_misaligned_pointers_rejected():
+    lib = _lib.lib()
+    cfg = _cfg()
+    ok = ctypes.c_void_p(256)
+    bad = ctypes.c_void_p(258)
+    assert lib.pisa_build_pyramid(ctypes.byref(cfg), None, ok, None) == 1
+    assert lib.pisa_build_pyramid(ctypes.byref(cfg), bad, ok, None) == 1
+    assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), ok, ok, ok, None, ok, None, None) == 1
+    assert lib.pisa_select(ctypes.byref(cfg), None, ok, ok, ok, None, ok, 1 << 30, None) == 1
+    assert lib.pisa_build_pyramid(None, ok, ok, None) == 1
+
+
+def test_select_workspace_too_small_rejected():
+    lib = _lib.lib()
+    cfg = _cfg(dtype=1)
+    need = lib.pisa_select_workspace_bytes(ctypes.byref(cfg))
+    assert need > 0
+    ok = ctypes.c_void_p(256)
+    assert lib.pisa_select(ctypes.byref(cfg), ok, ok, ok, ok, None, ok, need - 1, None) == 3
+    assert lib.pisa_select(ctypes.byref(cfg), ok, ok, ok, ok, None, None, need, None) == 3
+
+
+def test_decode_validation():
+    lib = _lib.lib()
+    dc = _lib.DecodeConfig(2, 300, 8, 2, 64, 32, 2, 4, 1, 0.0)
+    R = lib.pisa_decode_pyramid_rows(ctypes.byref(dc))
+    assert R == lib.pisa_pyramid_rows(300, 32)
+    bad = _lib.DecodeConfig(2, 0, 8, 2, 64, 32, 2, 4, 1, 0.0)
+    assert lib.pisa_decode_pyramid_rows(ctypes.byref(bad)) == 0
+    ok = ctypes.c_void_p(256)
+    assert lib.pisa_decode_append(ctypes.byref(dc), ok, ok, ok, ok, ok, ok, None, None) == 1  # status word required
+    assert lib.pisa_decode_step(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, ok, None, ok, None, ok, None) == 1

@@ -1,0 +1,97 @@
+"""GPU-vs-oracle parity of the prefill path through the C ABI: pyramid, PISA
+selection, flat selection and block-sparse attention, on the tiny fp32
+workload, on scaled-down copies of the bf16 workloads that span several tiles
+and a ragged tail, and on seeded row samples of the full-size workloads."""
+import numpy as np
+import pytest
+import torch
+
+import _parity as P
+import oracle as O
+from hierarchical_top_block_mean_b200 import api, workloads
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    workloads.PREFILL["tiny_noncausal_1k"],
+    workloads.PREFILL["tiny_noncausal_1k"].with_(name="tiny_causal_ragged", N=1000, causal=True, seed=1100),
+    workloads.PREFILL["tiny_noncausal_1k"].with_(name="tiny_bf16", dtype="bf16", seed=1200),
+    workloads.PREFILL["needle_16k"].with_(name="needle_3k_ragged", N=3000, n_needles=12, seed=2100),
+    workloads.PREFILL["clustered_64k"].with_(name="clustered_4k_G8", N=4160, H_q=16, H_kv=2, segment=512,
+                                             seed=3100),
+    workloads.PREFILL["needle_16k"].with_(name="f32_d128_ragged", N=2100, H_q=8, H_kv=2, dtype="f32",
+                                          n_needles=8, seed=2200),
+    workloads.PREFILL["clustered_64k"].with_(name="bf16_d64_C32_K5", N=2500, H_q=8, H_kv=4, d=64, C=32, K=5,
+                                             segment=256, seed=3200),
+    workloads.PREFILL["tiny_noncausal_1k"].with_(name="bf16_G1_noncausal", N=1500, H_q=2, H_kv=2, d=128, C=64,
+                                                 K=8, dtype="bf16", seed=1300),
+    workloads.PREFILL["tiny_noncausal_1k"].with_(name="bf16_G2_B2", B=2, N=777, H_q=4, H_kv=2, d=64, C=32, K=3,
+                                                 causal=True, dtype="bf16", seed=1400),
+]
+
+
+def _run(w, rows_per_head=None):
+    dev = torch.device("cuda")
+    x = workloads.prefill_inputs(w, device=dev)
+    q, k, v = x["q"], x["k"], x["v"]
+    pr = api.Problem.of(q, k, C=w.C, K=w.K, causal=w.causal)
+    p = api.Prefill(pr, dev)
+    p(q, k, v)
+    flat = api.select_flat(q, p.pyr, C=w.C, K=w.K, causal=w.causal, H_kv=w.H_kv)
+    torch.cuda.synchronize()
+    qh, kh, vh = P.host(q), P.host(k), P.host(v)
+    pyr_ref = P.check_pyramid(w, kh, P.host(p.pyr))
+    rows = P.sample_rows(w, rows_per_head, extra_t=[t for (t, _) in x["needles"]])
+    cfg = P.ocfg(w)
+    sel_ref, gap = O.select_rows(cfg, qh, kh, pyr_ref, rows)
+    sel_gpu = P.gather_rows(p.sel, rows)
+    n, n_ex, bad, bad_ex = P.compare_selection(w, sel_gpu, sel_ref, gap)
+    assert bad == 0, f"{w.name}: {bad} non-exempt selection mismatches of {n} rows ({n_ex} exempt)"
+    # Attention with the GPU's own selection, so selection differences cannot hide errors.
+    out_ref, lse_ref = O.attn_rows(cfg, qh, kh, vh, rows, sel_gpu)
+    err = P.check_attention(w, P.gather_out(w, p.out, rows), P.gather_lse(w, p.lse, rows), out_ref, lse_ref)
+    fsel_ref, fgap = O.select_flat_rows(cfg, qh, pyr_ref, rows)
+    fn, fex, fbad, _ = P.compare_selection(w, P.gather_rows(flat, rows), fsel_ref, fgap)
+    assert fbad == 0, f"{w.name}: flat selector {fbad} non-exempt mismatches of {fn}"
+    return dict(rows=n, exempt=n_ex, exempt_mismatch=bad_ex, attn_err=err, flat_exempt=fex)
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_prefill_parity_small(w):
+    r = _run(w)
+    print(w.name, r)
+
+
+def test_selection_output_format():
+    w = SMALL[1]
+    dev = torch.device("cuda")
+    x = workloads.prefill_inputs(w, device=dev)
+    out, lse, sel = api.prefill(x["q"], x["k"], x["v"], C=w.C, K=w.K, causal=w.causal)
+    s = P.host(sel).numpy()
+    for t in range(w.N):
+        nv = min(w.K, t // w.C + 1)
+        row = s[0, 0, t]
+        assert (row[:nv] >= 0).all() and (row[nv:] == -1).all()
+        assert (np.diff(row[:nv]) > 0).all()
+        assert row[:nv].max() <= t // w.C
+
+
+def test_large_K_prefill_equals_dense_attention():
+    # K >= number of leaves: everything is selected, attention is dense.
+    w = workloads.PREFILL["needle_16k"].with_(name="denseK", N=1000, H_q=8, H_kv=2, K=16, n_needles=0,
+                                              structure="iid", seed=9)
+    dev = torch.device("cuda")
+    x = workloads.prefill_inputs(w, device=dev)
+    out, lse, sel = api.prefill(x["q"], x["k"], x["v"], C=w.C, K=w.K, causal=True)
+    q, k, v = (x[n].float() for n in ("q", "k", "v"))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k.repeat_interleave(4, 1), v.repeat_interleave(4, 1),
+                                                           is_causal=True)
+    assert (out.float() - ref).abs().max().item() <= 2e-2
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,rows", [("needle_16k", None), ("clustered_64k", 2048), ("needle_256k", 1024)])
+def test_prefill_parity_full_size(name, rows):
+    w = workloads.PREFILL[name]
+    r = _run(w, rows)
+    print(name, r)
