@@ -1,12 +1,489 @@
+// Two-stage PISA selection for bf16 inputs (paper §Kernels, training and
+// prefill kernels):
+//   stage 1  router_kernel     one warp per (kv head, query): levels L..2 of
+//                              the coarse-to-fine search; candidate children
+//                              scored on tensor cores.
+//   grouping count (in stage 1), scan_kernel, scatter_kernel: a CSR of the
+//                              (query, candidate leaf) pairs keyed by leaf.
+//   stage 2  leaf_kernel       per leaf bucket: the C x d key tile is staged
+//                              in shared memory once and reused across tiles
+//                              of Q_tile = 4 queries x G_Q heads
+//                              ((Q_tile G_Q) x d . d x C on tensor cores),
+//                              then a per-head LSE over the keys and a sum
+//                              over the G_Q heads.
+//   final    final_kernel      top K of each row's leaf scores.
+//
+// Numerics: queries and keys are bf16, so q.k products are exact in a bf16
+// MMA with fp32 accumulation. Pyramid summaries are fp32; the router splits
+// each into bf16 hi + lo and issues two MMAs, which reproduces the fp32
+// summary to ~2^-16 relative.
+#include "dispatch.cuh"
+#include "mma.cuh"
+#include "rowops.cuh"
 #include "select2.cuh"
 
 namespace pisa {
 
-size_t select2_workspace_bytes(const PrefillArgs& a) { return 16; }
+namespace {
+
+constexpr int kRouterWarps = 4;
+constexpr int kPairsPerItem = 64;  // stage-2 work item: 16 query tiles of Q_tile = 4 pairs
+constexpr int kQTile = 4;
+constexpr int kLeafThreads = 128;
+
+// Workspace sections (all 256-byte aligned).
+struct Ws {
+  int32_t* cand;        // [rows][32] candidate leaves per row after stage 1 (-1 padded)
+  int32_t* ncand;       // [rows] candidates per row; -1 when stage 1 already wrote sel
+  float* score;         // [rows][32] leaf score of each candidate slot
+  int32_t* count;       // [buckets] pairs per (b, kv head, leaf)
+  int32_t* fill;        // [buckets] scatter cursors
+  int32_t* bucket_off;  // [buckets + 1] exclusive scan of count
+  int32_t* item_off;    // [buckets + 1] exclusive scan of ceil(count / kPairsPerItem)
+  uint32_t* pairs;      // [rows * 32] (t << 5 | slot), grouped by bucket
+};
+
+inline size_t al(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+size_t carve(const PrefillArgs& a, char* base, Ws* w) {
+  const size_t rows = static_cast<size_t>(a.B) * a.H_kv * a.N;
+  const size_t nb = static_cast<size_t>(a.B) * a.H_kv * level_size(a.N, a.C, 1);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + o : nullptr;
+    o += al(bytes);
+    return p;
+  };
+  Ws x;
+  x.cand = reinterpret_cast<int32_t*>(take(rows * 32 * 4));
+  x.ncand = reinterpret_cast<int32_t*>(take(rows * 4));
+  x.score = reinterpret_cast<float*>(take(rows * 32 * 4));
+  x.count = reinterpret_cast<int32_t*>(take(nb * 4));
+  x.fill = reinterpret_cast<int32_t*>(take(nb * 4));
+  x.bucket_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
+  x.item_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
+  x.pairs = reinterpret_cast<uint32_t*>(take(rows * 32 * 4));
+  if (w) *w = x;
+  return o;
+}
+
+__device__ inline bool usable(int64_t n, int C, int l, int64_t i, int64_t t, bool causal) {
+  if (i < 0 || i >= level_size(n, C, l)) return false;
+  return !causal || i * level_span(C, l) <= t;
+}
+
+// ---------------------------------------------------------------- stage 1
+template <int D, int G>
+__global__ void __launch_bounds__(kRouterWarps * 32)
+    router_kernel(const bf16* __restrict__ q, const float* __restrict__ pyr, Layout lay, PrefillArgs a, Ws ws,
+                  int32_t* __restrict__ sel, float* __restrict__ sel_score) {
+  __shared__ int tmp[kRouterWarps][32];
+  __shared__ int64_t off[kMaxLevels + 2];
+  load_offsets(lay, off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRouterWarps + warp;
+  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.N) return;
+  const int64_t n = a.N;
+  const int64_t bh = row / n, t = row % n;
+  const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
+  const bool causal = a.causal != 0;
+  const int C = a.C, K = a.K;
+  const float* P = pyr + bh * lay.R * D;
+  const float nanv = __int_as_float(0x7fffffff);
+
+  int l = num_levels(n, C);
+  while (l >= 1 && valid_count(n, C, l, t, causal) <= K) --l;
+  if (l < 1) {  // the leaf level itself has <= K usable blocks: keep them all
+    const int nv = static_cast<int>(valid_count(n, C, 1, t, causal));
+    if (lane < K) {
+      sel[row * K + lane] = lane < nv ? lane : -1;
+      if (sel_score) sel_score[row * K + lane] = nanv;
+    }
+    if (lane == 0) ws.ncand[row] = -1;
+    return;
+  }
+  int cand = lane < valid_count(n, C, l, t, causal) ? lane : -1;
+
+  if (l >= 2) {
+    // Query heads of the group as the B operand (columns = heads, zero padded to 8).
+    uint32_t qb[D / 16][2];
+    const int hd = gid < G ? gid : G - 1;
+    const bf16* qrow = q + ((b * a.H_q + h * G + hd) * n + t) * D + 4 * tig;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint2 u = *reinterpret_cast<const uint2*>(qrow + 16 * ks);
+      qb[ks][0] = gid < G ? u.x : 0u;
+      qb[ks][1] = gid < G ? u.y : 0u;
+    }
+    for (; l >= 2; --l) {
+      const int nc = warp_compact(cand, cand >= 0 && usable(n, C, l, cand, t, causal), tmp[warp]);
+      int nk = nc;
+      if (nc > K) {
+        // M-tile m holds candidates 8m .. 8m+7: row gid = first child, row gid + 8 = second.
+        float um[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          if (8 * m >= nc) break;
+          const int c = __shfl_sync(kFull, cand, 8 * m + gid);
+          const bool have = 8 * m + gid < nc;
+          const int64_t r0 = have ? 2 * static_cast<int64_t>(c) : 0;
+          const bool has1 = have && usable(n, C, l - 1, r0 + 1, t, causal);
+          const float* p0 = P + (off[l - 1] + r0) * D + 4 * tig;
+          const float* p1 = P + (off[l - 1] + (has1 ? r0 + 1 : r0)) * D + 4 * tig;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const float4 x0 = __ldg(reinterpret_cast<const float4*>(p0 + 16 * ks));
+            const float4 x1 = __ldg(reinterpret_cast<const float4*>(p1 + 16 * ks));
+            uint32_t hi[4], lo[4];
+            a_split(x0, x1, hi, lo);
+            mma_bf16(acc, hi, qb[ks][0], qb[ks][1]);
+            mma_bf16(acc, lo, qb[ks][0], qb[ks][1]);
+          }
+          // acc: [first child, head 2tig], [first, 2tig+1], [second, 2tig], [second, 2tig+1]
+          float u = 0.f;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (2 * tig + j < G) {
+              const float s0 = a.scale * acc[j];
+              u += has1 ? lse2(s0, a.scale * acc[2 + j]) : s0;
+            }
+          }
+          u += __shfl_xor_sync(kFull, u, 1);
+          u += __shfl_xor_sync(kFull, u, 2);
+          um[m] = have ? u : -INFINITY;
+        }
+        const int src = 4 * (lane & 7);
+        const float v0 = __shfl_sync(kFull, um[0], src), v1 = __shfl_sync(kFull, um[1], src);
+        const float v2 = __shfl_sync(kFull, um[2], src), v3 = __shfl_sync(kFull, um[3], src);
+        const int mm = lane >> 3;
+        float s = mm == 0 ? v0 : (mm == 1 ? v1 : (mm == 2 ? v2 : v3));
+        int idx = lane < nc ? cand : INT_MAX;
+        if (lane >= nc) s = -INFINITY;
+        warp_sort_desc(s, idx);
+        cand = idx;
+        nk = K;
+      }
+      const int parent = __shfl_sync(kFull, cand, lane >> 1);
+      cand = (lane >> 1) < nk ? 2 * parent + (lane & 1) : -1;
+    }
+  }
+  // Leaf-level candidates.
+  const int nc = warp_compact(cand, cand >= 0 && usable(n, C, 1, cand, t, causal), tmp[warp]);
+  if (nc <= K) {
+    int idx = lane < nc ? cand : INT_MAX;
+    warp_sort_asc(idx);
+    if (lane < K) {
+      sel[row * K + lane] = idx == INT_MAX ? -1 : idx;
+      if (sel_score) sel_score[row * K + lane] = nanv;
+    }
+    if (lane == 0) ws.ncand[row] = -1;
+    return;
+  }
+  ws.cand[row * 32 + lane] = lane < nc ? cand : -1;
+  if (lane == 0) ws.ncand[row] = nc;
+  if (lane < nc) atomicAdd(&ws.count[bh * level_size(n, C, 1) + cand], 1);
+}
+
+// ---------------------------------------------------------------- grouping
+// Exclusive scans of the pair counts (bucket offsets) and of the work items
+// per bucket, by one CTA.
+__global__ void __launch_bounds__(1024) scan_kernel(Ws ws, int nb) {
+  __shared__ int wsum[2][32];
+  __shared__ int carry[2];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry[0] = carry[1] = 0;
+  __syncthreads();
+  for (int base = 0; base < nb; base += 4096) {
+    int c[4], it[4], s0 = 0, s1 = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = base + threadIdx.x * 4 + j;
+      c[j] = i < nb ? ws.count[i] : 0;
+      it[j] = (c[j] + kPairsPerItem - 1) / kPairsPerItem;
+      s0 += c[j];
+      s1 += it[j];
+    }
+    int x0 = s0, x1 = s1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y0 = __shfl_up_sync(kFull, x0, o), y1 = __shfl_up_sync(kFull, x1, o);
+      if (lane >= o) {
+        x0 += y0;
+        x1 += y1;
+      }
+    }
+    if (lane == 31) {
+      wsum[0][warp] = x0;
+      wsum[1][warp] = x1;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int w0 = wsum[0][lane], w1 = wsum[1][lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y0 = __shfl_up_sync(kFull, w0, o), y1 = __shfl_up_sync(kFull, w1, o);
+        if (lane >= o) {
+          w0 += y0;
+          w1 += y1;
+        }
+      }
+      wsum[0][lane] = w0;
+      wsum[1][lane] = w1;
+    }
+    __syncthreads();
+    int e0 = carry[0] + (warp ? wsum[0][warp - 1] : 0) + x0 - s0;
+    int e1 = carry[1] + (warp ? wsum[1][warp - 1] : 0) + x1 - s1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = base + threadIdx.x * 4 + j;
+      if (i < nb) {
+        ws.bucket_off[i] = e0;
+        ws.item_off[i] = e1;
+      }
+      e0 += c[j];
+      e1 += it[j];
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) {
+      carry[0] = e0;
+      carry[1] = e1;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    ws.bucket_off[nb] = carry[0];
+    ws.item_off[nb] = carry[1];
+  }
+}
+
+// One thread per (row, slot): writes each pair into its leaf's bucket.
+__global__ void __launch_bounds__(256) scatter_kernel(Ws ws, int64_t rows, int N, int M1) {
+  const int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = x >> 5;
+  const int slot = static_cast<int>(x & 31);
+  if (row >= rows) return;
+  const int nc = ws.ncand[row];
+  if (slot >= nc) return;
+  const int leaf = ws.cand[row * 32 + slot];
+  const int64_t bh = row / N, t = row % N;
+  const int64_t bucket = bh * M1 + leaf;
+  const int pos = atomicAdd(&ws.fill[bucket], 1);
+  ws.pairs[ws.bucket_off[bucket] + pos] = (static_cast<uint32_t>(t) << 5) | static_cast<uint32_t>(slot);
+}
+
+// ---------------------------------------------------------------- stage 2
+// Key tile layout in shared memory: row r (one key) holds D bf16 as D/8
+// 16-byte chunks; chunk ch is stored at position ch ^ (r & 7) so that the
+// eight key rows read by one B-fragment load hit distinct banks.
+template <int D>
+__device__ inline uint2 key_frag(const bf16* tile, int r, int col) {
+  const int ch = col >> 3;
+  return *reinterpret_cast<const uint2*>(tile + r * D + ((ch ^ (r & 7)) << 3) + (col & 7));
+}
+
+template <int D, int G, int CC>
+__global__ void __launch_bounds__(kLeafThreads)
+    leaf_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, PrefillArgs a, Ws ws, int nb, int M1) {
+  constexpr int kMT = (kQTile * G + 15) / 16;  // 16-row M tiles per query tile
+  constexpr int kNT = CC / 8;                 // 8-key N tiles per leaf
+  constexpr int kKS = D / 16;                 // 16-wide k steps
+  __shared__ __align__(128) bf16 tile[CC * D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const bool causal = a.causal != 0;
+  const int total = ws.item_off[nb];
+  for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    int lo = 0, hi = nb;  // item_off[lo] <= item < item_off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (ws.item_off[mid] <= item) lo = mid;
+      else hi = mid;
+    }
+    const int bucket = lo;
+    const int chunk = item - ws.item_off[bucket];
+    const int p0 = ws.bucket_off[bucket] + chunk * kPairsPerItem;
+    const int p1 = min(p0 + kPairsPerItem, ws.bucket_off[bucket + 1]);
+    const int64_t bh = bucket / M1;
+    const int64_t leaf = bucket % M1;
+    const int64_t key0 = leaf * CC;
+    const int nkeys = static_cast<int>(min(static_cast<int64_t>(CC), a.N - key0));
+    const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
+    __syncthreads();  // the previous item's tile is no longer read
+    const bf16* ksrc = k + (bh * a.N + key0) * D;
+    for (int x = threadIdx.x; x < CC * D / 8; x += kLeafThreads) {
+      const int r = x / (D / 8), ch = x % (D / 8);
+      cp_async16(tile + r * D + ((ch ^ (r & 7)) << 3), ksrc + (r < nkeys ? r * D + ch * 8 : 0), r < nkeys ? 16 : 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    for (int tp = p0 + warp * kQTile; tp < p1; tp += 4 * kQTile) {
+      // The query tile: pair i of the tile is (t_i, slot_i); row r = i * G + head.
+      const uint32_t pw = lane < kQTile && tp + lane < p1 ? ws.pairs[tp + lane] : 0xffffffffu;
+      uint32_t a_reg[kMT][kKS][4];
+      int64_t t_row[kMT][2];
+      bool ok_row[kMT][2];
+#pragma unroll
+      for (int mt = 0; mt < kMT; ++mt) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int r = 16 * mt + gid + 8 * half;
+          const int pi = r / G, hd = r % G;
+          const uint32_t w = __shfl_sync(kFull, pw, pi < kQTile ? pi : 0);
+          const bool ok = r < kQTile * G && w != 0xffffffffu;
+          const int64_t tq = ok ? static_cast<int64_t>(w >> 5) : 0;
+          t_row[mt][half] = tq;
+          ok_row[mt][half] = ok;
+          const bf16* qp = q + ((b * a.H_q + h * G + hd) * a.N + tq) * D + 4 * tig;
+#pragma unroll
+          for (int ks = 0; ks < kKS; ++ks) {
+            uint2 u = make_uint2(0u, 0u);
+            if (ok) u = *reinterpret_cast<const uint2*>(qp + 16 * ks);
+            a_reg[mt][ks][half] = u.x;
+            a_reg[mt][ks][2 + half] = u.y;
+          }
+        }
+      }
+      float acc[kMT][kNT][4];
+#pragma unroll
+      for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < kKS; ++ks) {
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          const uint2 bb = key_frag<D>(tile, 8 * nt + gid, 16 * ks + 4 * tig);
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt) mma_bf16(acc[mt][nt], a_reg[mt][ks], bb.x, bb.y);
+        }
+      }
+      // Per (query, head) row: LSE over the usable keys of the leaf; then the
+      // sum over the G heads of each query (rows of one query are G
+      // consecutive rows, i.e. lanes that differ in the low bits of gid).
+#pragma unroll
+      for (int mt = 0; mt < kMT; ++mt) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int64_t tq = t_row[mt][half];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int kk = 8 * nt + 2 * tig + e;
+              const bool okk = kk < nkeys && (!causal || key0 + kk <= tq);
+              if (okk) mx = fmaxf(mx, a.scale * acc[mt][nt][2 * half + e]);
+            }
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+          float sum = 0.f;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int kk = 8 * nt + 2 * tig + e;
+              const bool okk = kk < nkeys && (!causal || key0 + kk <= tq);
+              if (okk) sum += expf(a.scale * acc[mt][nt][2 * half + e] - mx);
+            }
+          sum += __shfl_xor_sync(kFull, sum, 1);
+          sum += __shfl_xor_sync(kFull, sum, 2);
+          float u = ok_row[mt][half] ? mx + logf(sum) : 0.f;
+#pragma unroll
+          for (int o = 4; o < 4 * G; o <<= 1) u += __shfl_xor_sync(kFull, u, o);
+          // Writer: the first lane of each query's head group.
+          const int r = 16 * mt + gid + 8 * half;
+          const int pi = r / G;
+          const uint32_t w2 = __shfl_sync(kFull, pw, pi < kQTile ? pi : 0);
+          if (tig == 0 && (gid % G) == 0 && ok_row[mt][half]) {
+            const int64_t orow = bh * a.N + static_cast<int64_t>(w2 >> 5);
+            ws.score[orow * 32 + (w2 & 31)] = u;
+          }
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- final top-K
+__global__ void __launch_bounds__(256) final_kernel(PrefillArgs a, Ws ws, int32_t* __restrict__ sel,
+                                                    float* __restrict__ sel_score, int64_t rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= rows) return;
+  const int nc = ws.ncand[row];
+  if (nc < 0) return;  // stage 1 kept every usable leaf unscored and wrote sel
+  float s = lane < nc ? ws.score[row * 32 + lane] : -INFINITY;
+  int idx = lane < nc ? ws.cand[row * 32 + lane] : INT_MAX;
+  warp_sort_desc(s, idx);
+  if (lane >= a.K) {
+    idx = INT_MAX;
+    s = 0.f;
+  }
+  warp_sort_asc_kv(idx, s);
+  if (lane < a.K) {
+    sel[row * a.K + lane] = idx;
+    if (sel_score) sel_score[row * a.K + lane] = s;
+  }
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+size_t select2_workspace_bytes(const PrefillArgs& a) { return carve(a, nullptr, nullptr); }
 
 cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, const float* pyr, const Layout& lay,
-                           int32_t* sel, float* sel_score, void* ws, cudaStream_t st) {
-  return launch_select_rows(a, q, k, pyr, lay, sel, sel_score, st);
+                           int32_t* sel, float* sel_score, void* ws_ptr, cudaStream_t st) {
+  Ws ws;
+  carve(a, static_cast<char*>(ws_ptr), &ws);
+  const int64_t rows = static_cast<int64_t>(a.B) * a.H_kv * a.N;
+  const int M1 = static_cast<int>(level_size(a.N, a.C, 1));
+  const int nb = a.B * a.H_kv * M1;
+  cudaError_t e = cudaMemsetAsync(ws.count, 0, static_cast<size_t>(nb) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.fill, 0, static_cast<size_t>(nb) * 4, st);
+  if (e != cudaSuccess) return e;
+  const int G = a.H_q / a.H_kv;
+  e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
+    constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
+    router_kernel<D, GG><<<static_cast<unsigned>((rows + kRouterWarps - 1) / kRouterWarps), kRouterWarps * 32, 0,
+                           st>>>(static_cast<const bf16*>(q), pyr, lay, a, ws, sel, sel_score);
+    count_launch();
+    return cudaGetLastError();
+  });
+  if (e != cudaSuccess) return e;
+  scan_kernel<<<1, 1024, 0, st>>>(ws, nb);
+  count_launch();
+  scatter_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(ws, rows, a.N, M1);
+  count_launch();
+  const unsigned leaf_grid = static_cast<unsigned>(sm_count() * 4);
+  e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
+    constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
+    if (a.C == 64)
+      leaf_kernel<D, GG, 64><<<leaf_grid, kLeafThreads, 0, st>>>(static_cast<const bf16*>(q),
+                                                                  static_cast<const bf16*>(k), a, ws, nb, M1);
+    else
+      leaf_kernel<D, GG, 32><<<leaf_grid, kLeafThreads, 0, st>>>(static_cast<const bf16*>(q),
+                                                                  static_cast<const bf16*>(k), a, ws, nb, M1);
+    count_launch();
+    return cudaGetLastError();
+  });
+  if (e != cudaSuccess) return e;
+  final_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(a, ws, sel, sel_score, rows);
+  count_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace pisa
