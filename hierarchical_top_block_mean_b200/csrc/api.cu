@@ -59,6 +59,10 @@ DecodeArgs dargs_of(const pisa_decode_config* c) {
 }
 
 }  // namespace
+
+// Argument check shared with entry points defined in other files.
+pisa_status validate_prefill(const pisa_config* cfg) { return check_cfg(cfg); }
+
 }  // namespace pisa
 
 using namespace pisa;

@@ -146,6 +146,35 @@ pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float*
 pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
                                  const int32_t* sel, void* out, float* lse, void* stream);
 
+/*
+ * Size of the device array pisa_select_noalloc uses as its scratch: 64 MiB,
+ * reserved on every GPU that loads this library until the process exits.
+ */
+#define PISA_SELECT_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * pisa_select without a caller workspace. The paper has no counterpart: this
+ * is an interface for callers that cannot allocate device memory when they
+ * select, such as a plugin that its host framework hands only input and
+ * output buffers (no workspace hook), or a service whose memory pool owns the
+ * whole GPU. The selection (and every argument except the workspace) is that
+ * of pisa_select for bf16 inputs; the scratch lives in a library-owned device
+ * array of PISA_SELECT_NOALLOC_SCRATCH_BYTES.
+ *   - Returns PISA_ERR_WORKSPACE, enqueuing nothing, when the problem needs
+ *     more scratch than that (pisa_select_workspace_bytes(cfg) tells how much);
+ *     PISA_ERR_UNSUPPORTED for fp32 inputs, whose selection needs no scratch
+ *     (call pisa_select with ws = NULL).
+ *   - Calls no cudaMalloc or cudaFree and allocates nothing.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls in the process share the one array per device: calls whose
+ *     execution overlaps on the GPU (different streams, or different host
+ *     threads without ordering) race on it and give wrong selections. Order
+ *     them on one stream. Each call clears what it needs zeroed itself.
+ */
+pisa_status pisa_select_noalloc(const pisa_config* cfg, const void* q, const void* k, const float* pyr, int32_t* sel,
+                                float* sel_score, void* stream);
+
 /* ---------------------------------------------------------------- decode
  * §Kernels, decoding: the mean pyramid is cached; per new token only the
  * current leaf mean and its ancestor path are updated, and one fused kernel
