@@ -151,6 +151,8 @@ pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const vo
   if (s != PISA_OK) return s;
   if (!q || !k || !v || !sel || !out) return PISA_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return PISA_ERR_INVALID_ARGUMENT;
+  if (cfg->dtype == PISA_DTYPE_BF16)
+    return from_cuda(launch_attn_mma(args_of(cfg), q, k, v, sel, out, lse, as_stream(stream)));
   return from_cuda(launch_attn_rows(args_of(cfg), q, k, v, sel, out, lse, as_stream(stream)));
 }
 
