@@ -29,7 +29,7 @@ namespace {
 constexpr int kRouterWarps = 4;
 constexpr int kPairsPerItem = 64;  // stage-2 work item: 16 query tiles of Q_tile = 4 pairs
 constexpr int kQTile = 4;
-constexpr int kLeafThreads = 128;
+constexpr int kLeafThreads = 256;
 
 // Workspace sections (all 256-byte aligned).
 struct Ws {
@@ -41,6 +41,7 @@ struct Ws {
   int32_t* bucket_off;  // [buckets + 1] exclusive scan of count
   int32_t* item_off;    // [buckets + 1] exclusive scan of ceil(count / kPairsPerItem)
   uint32_t* pairs;      // [rows * 32] (t << 5 | slot), grouped by bucket
+  uint4* planes;        // [B*H_kv][R][D/4] pyramid rows as bf16 hi/lo: {hi x4, lo x4} per 4 elements
 };
 
 inline size_t al(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -63,6 +64,7 @@ size_t carve(const PrefillArgs& a, char* base, Ws* w) {
   x.bucket_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.item_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.pairs = reinterpret_cast<uint32_t*>(take(rows * 32 * 4));
+  x.planes = reinterpret_cast<uint4*>(take(static_cast<size_t>(a.B) * a.H_kv * make_layout(a.N, a.C).R * a.d * 4));
   if (w) *w = x;
   return o;
 }
@@ -70,6 +72,23 @@ size_t carve(const PrefillArgs& a, char* base, Ws* w) {
 __device__ inline bool usable(int64_t n, int C, int l, int64_t i, int64_t t, bool causal) {
   if (i < 0 || i >= level_size(n, C, l)) return false;
   return !causal || i * level_span(C, l) <= t;
+}
+
+// Pyramid rows (fp32) -> interleaved bf16 hi/lo chunks, so that the router
+// reads ready MMA operands: chunk c of a row holds hi(x[4c..4c+3]) then
+// lo(x[4c..4c+3]), with x - hi - lo below 2^-16 |x|.
+__global__ void __launch_bounds__(256) split_kernel(const float4* __restrict__ pyr, uint4* __restrict__ planes,
+                                                   int64_t n4) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 x = pyr[i];
+    float h[4], l[4];
+    split_bf16(x.x, h[0], l[0]);
+    split_bf16(x.y, h[1], l[1]);
+    split_bf16(x.z, h[2], l[2]);
+    split_bf16(x.w, h[3], l[3]);
+    planes[i] = make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]));
+  }
 }
 
 // ---------------------------------------------------------------- stage 1
@@ -89,7 +108,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
   const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
   const bool causal = a.causal != 0;
   const int C = a.C, K = a.K;
-  const float* P = pyr + bh * lay.R * D;
+  const uint4* PL = ws.planes + bh * lay.R * (D / 4);
   const float nanv = __int_as_float(0x7fffffff);
 
   int l = num_levels(n, C);
@@ -129,15 +148,19 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
           const bool have = 8 * m + gid < nc;
           const int64_t r0 = have ? 2 * static_cast<int64_t>(c) : 0;
           const bool has1 = have && usable(n, C, l - 1, r0 + 1, t, causal);
-          const float* p0 = P + (off[l - 1] + r0) * D + 4 * tig;
-          const float* p1 = P + (off[l - 1] + (has1 ? r0 + 1 : r0)) * D + 4 * tig;
+          const uint4* p0 = PL + (off[l - 1] + r0) * (D / 4) + tig;
+          const uint4* p1 = PL + (off[l - 1] + (has1 ? r0 + 1 : r0)) * (D / 4) + tig;
+          uint4 x0[D / 16], x1[D / 16];
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            x0[ks] = __ldg(p0 + 4 * ks);
+            x1[ks] = __ldg(p1 + 4 * ks);
+          }
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
-            const float4 x0 = __ldg(reinterpret_cast<const float4*>(p0 + 16 * ks));
-            const float4 x1 = __ldg(reinterpret_cast<const float4*>(p1 + 16 * ks));
-            uint32_t hi[4], lo[4];
-            a_split(x0, x1, hi, lo);
+            const uint32_t hi[4] = {x0[ks].x, x1[ks].x, x0[ks].y, x1[ks].y};
+            const uint32_t lo[4] = {x0[ks].z, x1[ks].z, x0[ks].w, x1[ks].w};
             mma_bf16(acc, hi, qb[ks][0], qb[ks][1]);
             mma_bf16(acc, lo, qb[ks][0], qb[ks][1]);
           }
@@ -283,128 +306,173 @@ __device__ inline uint2 key_frag(const bf16* tile, int r, int col) {
   return *reinterpret_cast<const uint2*>(tile + r * D + ((ch ^ (r & 7)) << 3) + (col & 7));
 }
 
+// Copies the C x D key tile of one leaf into shared memory (swizzled as
+// key_frag expects); rows past the sequence end are zero-filled.
+template <int D, int CC>
+__device__ inline void load_key_tile(bf16* tile, const bf16* __restrict__ ksrc, int nkeys) {
+  for (int x = threadIdx.x; x < CC * D / 8; x += blockDim.x) {
+    const int r = x / (D / 8), ch = x % (D / 8);
+    cp_async16(tile + r * D + ((ch ^ (r & 7)) << 3), ksrc + (r < nkeys ? r * D + ch * 8 : 0), r < nkeys ? 16 : 0);
+  }
+  cp_async_commit();
+}
+
+// Stage 2. Each CTA owns a contiguous range of work items (64 pairs each,
+// ordered by bucket). Consecutive items of one bucket share the key tile in
+// shared memory; the next bucket's tile is prefetched (double buffer) while
+// the current one is scored. A warp scores one 16-row M tile at a time: the
+// 16 / G queries of a query tile (Q_tile = 4 queries x G heads is split into
+// passes of at most 16 rows), against all C keys of the tile.
 template <int D, int G, int CC>
-__global__ void __launch_bounds__(kLeafThreads)
+__global__ void __launch_bounds__(kLeafThreads, 2)
     leaf_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, PrefillArgs a, Ws ws, int nb, int M1) {
-  constexpr int kMT = (kQTile * G + 15) / 16;  // 16-row M tiles per query tile
   constexpr int kNT = CC / 8;                 // 8-key N tiles per leaf
   constexpr int kKS = D / 16;                 // 16-wide k steps
-  __shared__ __align__(128) bf16 tile[CC * D];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kP = G >= 8 ? 2 : kQTile;     // queries per 16-row M tile
+  constexpr float kLog2e = 1.4426950408889634f;
+  __shared__ __align__(128) bf16 tiles[2][CC * D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const bool causal = a.causal != 0;
+  const float sl2 = a.scale * kLog2e;
+
   const int total = ws.item_off[nb];
-  for (int item = blockIdx.x; item < total; item += gridDim.x) {
-    int lo = 0, hi = nb;  // item_off[lo] <= item < item_off[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (ws.item_off[mid] <= item) lo = mid;
-      else hi = mid;
+  const int per = (total + gridDim.x - 1) / gridDim.x;
+  const int i0 = blockIdx.x * per;
+  const int i1 = min(i0 + per, total);
+  if (i0 >= i1) return;
+  int lo = 0, hi = nb;  // bucket of i0: item_off[lo] <= i0 < item_off[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (ws.item_off[mid] <= i0) lo = mid;
+    else hi = mid;
+  }
+  int bucket = lo;
+  int buf = 0;
+  auto key_src = [&](int bk, int& nkeys) {
+    const int64_t bh = bk / M1, leaf = bk % M1;
+    nkeys = static_cast<int>(min(static_cast<int64_t>(CC), a.N - leaf * CC));
+    return k + (bh * a.N + leaf * CC) * D;
+  };
+  {
+    int nk;
+    const bf16* src = key_src(bucket, nk);
+    load_key_tile<D, CC>(tiles[0], src, nk);
+  }
+  while (true) {
+    // Items of this bucket inside [i0, i1) and their pairs.
+    const int it_lo = max(ws.item_off[bucket], i0);
+    const int it_hi = min(ws.item_off[bucket + 1], i1);
+    const int base = ws.bucket_off[bucket];
+    const int p_lo = base + (it_lo - ws.item_off[bucket]) * kPairsPerItem;
+    const int p_hi = min(base + (it_hi - ws.item_off[bucket]) * kPairsPerItem, ws.bucket_off[bucket + 1]);
+    // Next bucket with work inside the range: prefetch its tile.
+    int next = -1;
+    if (it_hi < i1) {
+      next = bucket + 1;
+      while (ws.item_off[next + 1] <= it_hi) ++next;  // skip buckets without items
+      int nk;
+      const bf16* src = key_src(next, nk);
+      load_key_tile<D, CC>(tiles[buf ^ 1], src, nk);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    const int bucket = lo;
-    const int chunk = item - ws.item_off[bucket];
-    const int p0 = ws.bucket_off[bucket] + chunk * kPairsPerItem;
-    const int p1 = min(p0 + kPairsPerItem, ws.bucket_off[bucket + 1]);
-    const int64_t bh = bucket / M1;
-    const int64_t leaf = bucket % M1;
-    const int64_t key0 = leaf * CC;
-    const int nkeys = static_cast<int>(min(static_cast<int64_t>(CC), a.N - key0));
-    const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
-    __syncthreads();  // the previous item's tile is no longer read
-    const bf16* ksrc = k + (bh * a.N + key0) * D;
-    for (int x = threadIdx.x; x < CC * D / 8; x += kLeafThreads) {
-      const int r = x / (D / 8), ch = x % (D / 8);
-      cp_async16(tile + r * D + ((ch ^ (r & 7)) << 3), ksrc + (r < nkeys ? r * D + ch * 8 : 0), r < nkeys ? 16 : 0);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
     __syncthreads();
 
-    for (int tp = p0 + warp * kQTile; tp < p1; tp += 4 * kQTile) {
-      // The query tile: pair i of the tile is (t_i, slot_i); row r = i * G + head.
-      const uint32_t pw = lane < kQTile && tp + lane < p1 ? ws.pairs[tp + lane] : 0xffffffffu;
-      uint32_t a_reg[kMT][kKS][4];
-      int64_t t_row[kMT][2];
-      bool ok_row[kMT][2];
+    const bf16* tile = tiles[buf];
+    const int64_t bh = bucket / M1;
+    const int64_t key0 = static_cast<int64_t>(bucket % M1) * CC;
+    const int nkeys = static_cast<int>(min(static_cast<int64_t>(CC), a.N - key0));
+    const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
+    const bf16* qbase = q + ((b * a.H_q + h * G) * a.N) * D + 4 * tig;
+    for (int u0 = p_lo + warp * kP; u0 < p_hi; u0 += nwarps * kP) {
+      const uint32_t pw = (lane < kP && u0 + lane < p_hi) ? ws.pairs[u0 + lane] : 0xffffffffu;
+      uint32_t a_reg[kKS][4];
+      int nvk[2];
+      bool ok[2];
 #pragma unroll
-      for (int mt = 0; mt < kMT; ++mt) {
+      for (int half = 0; half < 2; ++half) {
+        const int r = gid + 8 * half;
+        const int pi = r / G, hd = r % G;
+        const uint32_t w = __shfl_sync(kFull, pw, pi < kP ? pi : 0);
+        ok[half] = pi < kP && w != 0xffffffffu;
+        const int64_t tq = ok[half] ? static_cast<int64_t>(w >> 5) : 0;
+        // usable keys of the tile for this query: [0, nvk)
+        int64_t nv = nkeys;
+        if (causal) nv = min(nv, tq - key0 + 1);
+        nvk[half] = static_cast<int>(max(nv, static_cast<int64_t>(0)));
+        const bf16* qp = qbase + (static_cast<int64_t>(hd) * a.N + tq) * D;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int r = 16 * mt + gid + 8 * half;
-          const int pi = r / G, hd = r % G;
-          const uint32_t w = __shfl_sync(kFull, pw, pi < kQTile ? pi : 0);
-          const bool ok = r < kQTile * G && w != 0xffffffffu;
-          const int64_t tq = ok ? static_cast<int64_t>(w >> 5) : 0;
-          t_row[mt][half] = tq;
-          ok_row[mt][half] = ok;
-          const bf16* qp = q + ((b * a.H_q + h * G + hd) * a.N + tq) * D + 4 * tig;
-#pragma unroll
-          for (int ks = 0; ks < kKS; ++ks) {
-            uint2 u = make_uint2(0u, 0u);
-            if (ok) u = *reinterpret_cast<const uint2*>(qp + 16 * ks);
-            a_reg[mt][ks][half] = u.x;
-            a_reg[mt][ks][2 + half] = u.y;
-          }
+        for (int ks = 0; ks < kKS; ++ks) {
+          uint2 uu = make_uint2(0u, 0u);
+          if (ok[half]) uu = *reinterpret_cast<const uint2*>(qp + 16 * ks);
+          a_reg[ks][half] = uu.x;
+          a_reg[ks][2 + half] = uu.y;
         }
       }
-      float acc[kMT][kNT][4];
+      float acc[kNT][4];
 #pragma unroll
-      for (int mt = 0; mt < kMT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+      for (int nt = 0; nt < kNT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
       for (int ks = 0; ks < kKS; ++ks) {
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) {
           const uint2 bb = key_frag<D>(tile, 8 * nt + gid, 16 * ks + 4 * tig);
-#pragma unroll
-          for (int mt = 0; mt < kMT; ++mt) mma_bf16(acc[mt][nt], a_reg[mt][ks], bb.x, bb.y);
+          mma_bf16(acc[nt], a_reg[ks], bb.x, bb.y);
         }
       }
-      // Per (query, head) row: LSE over the usable keys of the leaf; then the
-      // sum over the G heads of each query (rows of one query are G
-      // consecutive rows, i.e. lanes that differ in the low bits of gid).
+      // Per (query, head) row: LSE over the usable keys, in log2 units.
 #pragma unroll
-      for (int mt = 0; mt < kMT; ++mt) {
+      for (int half = 0; half < 2; ++half) {
+        const int nv = nvk[half];
+        float mx = -INFINITY;
+        if (nv >= CC) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int64_t tq = t_row[mt][half];
-          float mx = -INFINITY;
-#pragma unroll
-          for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int kk = 8 * nt + 2 * tig + e;
-              const bool okk = kk < nkeys && (!causal || key0 + kk <= tq);
-              if (okk) mx = fmaxf(mx, a.scale * acc[mt][nt][2 * half + e]);
-            }
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-          float sum = 0.f;
+          for (int nt = 0; nt < kNT; ++nt) mx = fmaxf(mx, fmaxf(acc[nt][2 * half], acc[nt][2 * half + 1]));
+        } else {
 #pragma unroll
           for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int kk = 8 * nt + 2 * tig + e;
-              const bool okk = kk < nkeys && (!causal || key0 + kk <= tq);
-              if (okk) sum += expf(a.scale * acc[mt][nt][2 * half + e] - mx);
-            }
-          sum += __shfl_xor_sync(kFull, sum, 1);
-          sum += __shfl_xor_sync(kFull, sum, 2);
-          float u = ok_row[mt][half] ? mx + logf(sum) : 0.f;
+            for (int e = 0; e < 2; ++e)
+              if (8 * nt + 2 * tig + e < nv) mx = fmaxf(mx, acc[nt][2 * half + e]);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const float mxs = mx * sl2;
+        float sum = 0.f;
+        if (nv >= CC) {
 #pragma unroll
-          for (int o = 4; o < 4 * G; o <<= 1) u += __shfl_xor_sync(kFull, u, o);
-          // Writer: the first lane of each query's head group.
-          const int r = 16 * mt + gid + 8 * half;
-          const int pi = r / G;
-          const uint32_t w2 = __shfl_sync(kFull, pw, pi < kQTile ? pi : 0);
-          if (tig == 0 && (gid % G) == 0 && ok_row[mt][half]) {
-            const int64_t orow = bh * a.N + static_cast<int64_t>(w2 >> 5);
-            ws.score[orow * 32 + (w2 & 31)] = u;
-          }
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) sum += exp2f(fmaf(acc[nt][2 * half + e], sl2, -mxs));
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              if (8 * nt + 2 * tig + e < nv) sum += exp2f(fmaf(acc[nt][2 * half + e], sl2, -mxs));
+        }
+        sum += __shfl_xor_sync(kFull, sum, 1);
+        sum += __shfl_xor_sync(kFull, sum, 2);
+        float u = ok[half] ? mx * a.scale + logf(sum) : 0.f;
+        // Sum over the G heads of each query: rows r .. r + G - 1 sit in
+        // lanes that differ in the low log2(G) bits of gid.
+#pragma unroll
+        for (int o = 4; o < 4 * G; o <<= 1) u += __shfl_xor_sync(kFull, u, o);
+        const int r = gid + 8 * half;
+        const int pi = r / G;
+        const uint32_t w = __shfl_sync(kFull, pw, pi < kP ? pi : 0);
+        if (tig == 0 && (gid % G) == 0 && ok[half]) {
+          const int64_t orow = bh * a.N + static_cast<int64_t>(w >> 5);
+          ws.score[orow * 32 + (w & 31)] = u;
         }
       }
     }
+    if (next < 0) break;
+    __syncthreads();  // every warp is done with tiles[buf] before it is refilled
+    bucket = next;
+    buf ^= 1;
   }
 }
 
@@ -456,6 +524,14 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.fill, 0, static_cast<size_t>(nb) * 4, st);
   if (e != cudaSuccess) return e;
   const int G = a.H_q / a.H_kv;
+  {
+    const int64_t n4 = static_cast<int64_t>(a.B) * a.H_kv * lay.R * a.d / 4;
+    const int64_t gb = (n4 + 255) / 256;
+    const unsigned g = static_cast<unsigned>(gb < sm_count() * 16 ? gb : sm_count() * 16);
+    split_kernel<<<g, 256, 0, st>>>(reinterpret_cast<const float4*>(pyr), ws.planes, n4);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
     constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
     router_kernel<D, GG><<<static_cast<unsigned>((rows + kRouterWarps - 1) / kRouterWarps), kRouterWarps * 32, 0,
@@ -468,7 +544,7 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   count_launch();
   scatter_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(ws, rows, a.N, M1);
   count_launch();
-  const unsigned leaf_grid = static_cast<unsigned>(sm_count() * 4);
+  const unsigned leaf_grid = static_cast<unsigned>(sm_count() * 2);
   e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
     constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
     if (a.C == 64)
