@@ -142,6 +142,7 @@ pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float*
   if (s != PISA_OK) return s;
   if (!q || !pyr || !sel || !aligned16(q) || !aligned16(pyr) || !aligned16(sel)) return PISA_ERR_INVALID_ARGUMENT;
   const Layout lay = make_layout(cfg->N, cfg->C);
+  if (cfg->dtype == PISA_DTYPE_BF16) return from_cuda(launch_flat_mma(args_of(cfg), q, pyr, lay.R, sel, as_stream(stream)));
   return from_cuda(launch_flat_rows(args_of(cfg), q, pyr, lay.R, sel, as_stream(stream)));
 }
 

@@ -30,6 +30,9 @@ cudaError_t launch_flat_rows(const PrefillArgs& a, const void* q, const float* p
 cudaError_t launch_attn_mma(const PrefillArgs& a, const void* q, const void* k, const void* v, const int32_t* sel,
                             void* out, float* lse, cudaStream_t st);
 
+cudaError_t launch_flat_mma(const PrefillArgs& a, const void* q, const float* pyr, int64_t R, int32_t* sel,
+                            cudaStream_t st);
+
 // ---- decode
 cudaError_t launch_decode_append(const DecodeArgs& a, const Layout& lay, const void* k_new, const void* v_new,
                                  void* k_cache, void* v_cache, float* pyr, int32_t* len, int32_t* status,
