@@ -179,8 +179,11 @@ pisa_status pisa_decode_append(const pisa_decode_config* cfg, const void* k_new,
   if (!k_new || !v_new || !k_cache || !v_cache || !pyr || !len || !status) return PISA_ERR_INVALID_ARGUMENT;
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(pyr)) return PISA_ERR_INVALID_ARGUMENT;
   const Layout lay = make_layout(cfg->cap, cfg->C);
-  return from_cuda(launch_decode_append(dargs_of(cfg), lay, k_new, v_new, k_cache, v_cache, pyr, len, status,
-                                        as_stream(stream)));
+  const DecodeArgs a = dargs_of(cfg);
+  if (decode_fused_supported(a))
+    return from_cuda(launch_decode_fused(a, lay, 1, nullptr, k_new, v_new, k_cache, v_cache, pyr, len, nullptr, nullptr,
+                                         nullptr, status, as_stream(stream)));
+  return from_cuda(launch_decode_append(a, lay, k_new, v_new, k_cache, v_cache, pyr, len, status, as_stream(stream)));
 }
 
 pisa_status pisa_decode_select(const pisa_decode_config* cfg, const void* q_new, const void* k_cache,
@@ -190,8 +193,14 @@ pisa_status pisa_decode_select(const pisa_decode_config* cfg, const void* q_new,
   if (!q_new || !k_cache || !pyr || !len || !sel) return PISA_ERR_INVALID_ARGUMENT;
   if (!aligned16(q_new) || !aligned16(k_cache) || !aligned16(pyr)) return PISA_ERR_INVALID_ARGUMENT;
   const Layout lay = make_layout(cfg->cap, cfg->C);
-  return from_cuda(launch_decode_rows(dargs_of(cfg), lay, 1, q_new, k_cache, nullptr, pyr, len, sel, nullptr,
-                                      nullptr, as_stream(stream)));
+  const DecodeArgs a = dargs_of(cfg);
+  if (decode_fused_supported(a))
+    return from_cuda(launch_decode_fused(a, lay, 2, q_new, nullptr, nullptr, const_cast<void*>(k_cache),
+                                         const_cast<void*>(k_cache), const_cast<float*>(pyr),
+                                         const_cast<int32_t*>(len), sel, nullptr, nullptr, nullptr,
+                                         as_stream(stream)));
+  return from_cuda(launch_decode_rows(a, lay, 1, q_new, k_cache, nullptr, pyr, len, sel, nullptr, nullptr,
+                                      as_stream(stream)));
 }
 
 pisa_status pisa_decode_attn(const pisa_decode_config* cfg, const void* q_new, const void* k_cache,
@@ -202,8 +211,13 @@ pisa_status pisa_decode_attn(const pisa_decode_config* cfg, const void* q_new, c
   if (!q_new || !k_cache || !v_cache || !len || !sel || !out) return PISA_ERR_INVALID_ARGUMENT;
   if (!aligned16(q_new) || !aligned16(k_cache) || !aligned16(v_cache)) return PISA_ERR_INVALID_ARGUMENT;
   const Layout lay = make_layout(cfg->cap, cfg->C);
-  return from_cuda(launch_decode_rows(dargs_of(cfg), lay, 2, q_new, k_cache, v_cache, nullptr, len,
-                                      const_cast<int32_t*>(sel), out, lse, as_stream(stream)));
+  const DecodeArgs a = dargs_of(cfg);
+  if (decode_fused_supported(a))
+    return from_cuda(launch_decode_fused(a, lay, 4, q_new, nullptr, nullptr, const_cast<void*>(k_cache),
+                                         const_cast<void*>(v_cache), nullptr, const_cast<int32_t*>(len),
+                                         const_cast<int32_t*>(sel), out, lse, nullptr, as_stream(stream)));
+  return from_cuda(launch_decode_rows(a, lay, 2, q_new, k_cache, v_cache, nullptr, len, const_cast<int32_t*>(sel),
+                                      out, lse, as_stream(stream)));
 }
 
 pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, const void* k_new, const void* v_new,
@@ -217,6 +231,9 @@ pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, c
     return PISA_ERR_INVALID_ARGUMENT;
   const Layout lay = make_layout(cfg->cap, cfg->C);
   const DecodeArgs a = dargs_of(cfg);
+  if (decode_fused_supported(a))
+    return from_cuda(launch_decode_fused(a, lay, 7, q_new, k_new, v_new, k_cache, v_cache, pyr, len, sel, out, lse,
+                                         status, as_stream(stream)));
   cudaError_t e = launch_decode_append(a, lay, k_new, v_new, k_cache, v_cache, pyr, len, status, as_stream(stream));
   if (e != cudaSuccess) return PISA_ERR_CUDA;
   return from_cuda(

@@ -43,4 +43,10 @@ cudaError_t launch_decode_rows(const DecodeArgs& a, const Layout& lay, int mode,
                                const void* k_cache, const void* v_cache, const float* pyr, const int32_t* len,
                                int32_t* sel, void* out, float* lse, cudaStream_t st);
 
+// Fused decode (bf16, H_kv <= 8, G_Q <= 8). mode bits: 1 append, 2 select, 4 attend.
+bool decode_fused_supported(const DecodeArgs& a);
+cudaError_t launch_decode_fused(const DecodeArgs& a, const Layout& lay, int mode, const void* q_new,
+                                const void* k_new, const void* v_new, void* k_cache, void* v_cache, float* pyr,
+                                int32_t* len, int32_t* sel, void* out, float* lse, int32_t* status, cudaStream_t st);
+
 }  // namespace pisa
