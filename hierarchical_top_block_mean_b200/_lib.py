@@ -45,6 +45,7 @@ SIGNATURES = {
     "pisa_status_string": (ctypes.c_char_p, [_i32]),
     "pisa_version": (_i32, []),
     "pisa_launch_count": (ctypes.c_uint64, []),
+    "pisa_device_faults": (ctypes.c_uint64, []),
     "pisa_pyramid_geometry": (_i32, [_i64, _i32, _i32, ctypes.POINTER(_i32), _p]),
     "pisa_pyramid_rows": (_i64, [_i64, _i32]),
     "pisa_build_pyramid": (_i32, [_PC, _p, _p, _p]),

@@ -42,6 +42,11 @@ def launch_count() -> int:
     return int(_lib.lib().pisa_launch_count())
 
 
+def device_faults() -> int:
+    """Bounded device waits that ran out of time on the current device (synchronises)."""
+    return int(_lib.lib().pisa_device_faults())
+
+
 def pyramid_geometry(N: int, C: int, g: int = 2):
     """(L, offsets): level l (1..L) occupies rows offsets[l-1]:offsets[l]."""
     L = ctypes.c_int32()

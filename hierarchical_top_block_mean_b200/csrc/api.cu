@@ -7,6 +7,7 @@
 #include "kernels.cuh"
 #include "pyramid.cuh"
 #include "select2.cuh"
+#include "tma.cuh"
 
 namespace pisa {
 
@@ -85,6 +86,13 @@ const char* pisa_status_string(int32_t status) {
 int32_t pisa_version(void) { return 100; }
 
 uint64_t pisa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+uint64_t pisa_device_faults(void) {
+  unsigned long long* p = wait_fault_counter();
+  unsigned long long v = 0;
+  if (!p || cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return UINT64_MAX;
+  return v;
+}
 
 pisa_status pisa_pyramid_geometry(int64_t N, int32_t C, int32_t g, int32_t* num_levels_out, int64_t* level_offsets) {
   if (N < 1 || C < 1 || g != 2 || !num_levels_out) return PISA_ERR_INVALID_ARGUMENT;

@@ -26,7 +26,7 @@ constexpr int kChunk = 64;                // leaves per shared-memory chunk
 template <int D>
 __device__ inline uint2 plane_frag(const bf16* plane, int r, int col) {
   const int ch = col >> 3;
-  return *reinterpret_cast<const uint2*>(plane + r * D + ((ch ^ (r & 7)) << 3) + (col & 7));
+  return *reinterpret_cast<const uint2*>(plane + r * D + ((ch ^ ((r & 3) << 1)) << 3) + (col & 7));
 }
 
 template <int D, int G>
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kFlatWarps * 32, 2)
       float hh[8], ll[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) split_bf16(f[j], hh[j], ll[j]);
-      const int off = r * D + ((ch ^ (r & 7)) << 3);
+      const int off = r * D + ((ch ^ ((r & 3) << 1)) << 3);
       *reinterpret_cast<uint4*>(phi + off) =
           make_uint4(pack_bf16(hh[0], hh[1]), pack_bf16(hh[2], hh[3]), pack_bf16(hh[4], hh[5]), pack_bf16(hh[6], hh[7]));
       *reinterpret_cast<uint4*>(plo + off) =

@@ -42,13 +42,28 @@ struct Ws {
   int32_t* item_off;    // [buckets + 1] exclusive scan of ceil(count / kPairsPerItem)
   uint32_t* pairs;      // [rows * 32] (t << 5 | slot), grouped by bucket
   uint4* planes;        // [B*H_kv][R][D/4] pyramid rows as bf16 hi/lo: {hi x4, lo x4} per 4 elements
+  int32_t* item_bucket; // [items] bucket of each stage-2 work item
+  int win_shift;        // queries are bucketed by window t >> win_shift
+  int nwin;             // windows per (b, kv head)
 };
+
+// Query window of the stage-2 buckets: about 32 MB of one kv head's queries
+// (W x G_Q x d x 2 bytes), so that a window's queries stay L2-resident while
+// all CTAs score its buckets.
+inline int window_shift(const PrefillArgs& a) {
+  const int64_t per_query = static_cast<int64_t>(a.H_q / a.H_kv) * a.d * 2;
+  int sh = 6;
+  while ((int64_t{1} << (sh + 1)) * per_query <= (int64_t{32} << 20) && sh < 30) ++sh;
+  return sh;
+}
 
 inline size_t al(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 size_t carve(const PrefillArgs& a, char* base, Ws* w) {
   const size_t rows = static_cast<size_t>(a.B) * a.H_kv * a.N;
-  const size_t nb = static_cast<size_t>(a.B) * a.H_kv * level_size(a.N, a.C, 1);
+  const int sh = window_shift(a);
+  const int nwin = static_cast<int>((static_cast<int64_t>(a.N) + (int64_t{1} << sh) - 1) >> sh);
+  const size_t nb = static_cast<size_t>(a.B) * a.H_kv * nwin * level_size(a.N, a.C, 1);
   size_t o = 0;
   auto take = [&](size_t bytes) {
     char* p = base ? base + o : nullptr;
@@ -65,6 +80,9 @@ size_t carve(const PrefillArgs& a, char* base, Ws* w) {
   x.item_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.pairs = reinterpret_cast<uint32_t*>(take(rows * 32 * 4));
   x.planes = reinterpret_cast<uint4*>(take(static_cast<size_t>(a.B) * a.H_kv * make_layout(a.N, a.C).R * a.d * 4));
+  x.item_bucket = reinterpret_cast<int32_t*>(take((rows * 32 / kPairsPerItem + nb + 1) * 4));
+  x.win_shift = sh;
+  x.nwin = nwin;
   if (w) *w = x;
   return o;
 }
@@ -206,7 +224,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
   }
   ws.cand[row * 32 + lane] = lane < nc ? cand : -1;
   if (lane == 0) ws.ncand[row] = nc;
-  if (lane < nc) atomicAdd(&ws.count[bh * level_size(n, C, 1) + cand], 1);
+  if (lane < nc) atomicAdd(&ws.count[(bh * ws.nwin + (t >> ws.win_shift)) * level_size(n, C, 1) + cand], 1);
 }
 
 // ---------------------------------------------------------------- grouping
@@ -291,19 +309,27 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ws ws, int64_t rows, int N
   if (slot >= nc) return;
   const int leaf = ws.cand[row * 32 + slot];
   const int64_t bh = row / N, t = row % N;
-  const int64_t bucket = bh * M1 + leaf;
+  const int64_t bucket = (bh * ws.nwin + (t >> ws.win_shift)) * M1 + leaf;
   const int pos = atomicAdd(&ws.fill[bucket], 1);
   ws.pairs[ws.bucket_off[bucket] + pos] = (static_cast<uint32_t>(t) << 5) | static_cast<uint32_t>(slot);
 }
 
+// Item -> bucket map: one thread per bucket writes its items' entries.
+__global__ void __launch_bounds__(256) itemize_kernel(Ws ws, int nb) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= nb) return;
+  for (int i = ws.item_off[b]; i < ws.item_off[b + 1]; ++i) ws.item_bucket[i] = b;
+}
+
 // ---------------------------------------------------------------- stage 2
 // Key tile layout in shared memory: row r (one key) holds D bf16 as D/8
-// 16-byte chunks; chunk ch is stored at position ch ^ (r & 7) so that the
-// eight key rows read by one B-fragment load hit distinct banks.
+// 16-byte chunks; chunk ch is stored at position ch ^ 2 (r & 3). A 64-bit
+// fragment load is served per half-warp (rows gid = 0..3 or 4..7, two
+// chunks each); this swizzle puts those eight 8-byte reads in distinct banks.
 template <int D>
 __device__ inline uint2 key_frag(const bf16* tile, int r, int col) {
   const int ch = col >> 3;
-  return *reinterpret_cast<const uint2*>(tile + r * D + ((ch ^ (r & 7)) << 3) + (col & 7));
+  return *reinterpret_cast<const uint2*>(tile + r * D + ((ch ^ ((r & 3) << 1)) << 3) + (col & 7));
 }
 
 // Copies the C x D key tile of one leaf into shared memory (swizzled as
@@ -312,7 +338,7 @@ template <int D, int CC>
 __device__ inline void load_key_tile(bf16* tile, const bf16* __restrict__ ksrc, int nkeys) {
   for (int x = threadIdx.x; x < CC * D / 8; x += blockDim.x) {
     const int r = x / (D / 8), ch = x % (D / 8);
-    cp_async16(tile + r * D + ((ch ^ (r & 7)) << 3), ksrc + (r < nkeys ? r * D + ch * 8 : 0), r < nkeys ? 16 : 0);
+    cp_async16(tile + r * D + ((ch ^ ((r & 3) << 1)) << 3), ksrc + (r < nkeys ? r * D + ch * 8 : 0), r < nkeys ? 16 : 0);
   }
   cp_async_commit();
 }
@@ -336,41 +362,31 @@ __global__ void __launch_bounds__(kLeafThreads, 2)
   const bool causal = a.causal != 0;
   const float sl2 = a.scale * kLog2e;
 
+  // Items are walked grid-strided, so that at any time all CTAs work on
+  // neighbouring buckets (the same query window) and the window's queries
+  // stay in L2. A tile is reused when the next item has the same bucket.
   const int total = ws.item_off[nb];
-  const int per = (total + gridDim.x - 1) / gridDim.x;
-  const int i0 = blockIdx.x * per;
-  const int i1 = min(i0 + per, total);
-  if (i0 >= i1) return;
-  int lo = 0, hi = nb;  // bucket of i0: item_off[lo] <= i0 < item_off[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (ws.item_off[mid] <= i0) lo = mid;
-    else hi = mid;
-  }
-  int bucket = lo;
-  int buf = 0;
+  int item = blockIdx.x;
+  if (item >= total) return;
+  const int64_t bucket_span = static_cast<int64_t>(ws.nwin) * M1;  // buckets per (b, kv head)
   auto key_src = [&](int bk, int& nkeys) {
-    const int64_t bh = bk / M1, leaf = bk % M1;
+    const int64_t bhh = bk / bucket_span, leaf = bk % M1;
     nkeys = static_cast<int>(min(static_cast<int64_t>(CC), a.N - leaf * CC));
-    return k + (bh * a.N + leaf * CC) * D;
+    return k + (bhh * a.N + leaf * CC) * D;
   };
+  int bucket = ws.item_bucket[item];
+  int buf = 0;
   {
     int nk;
     const bf16* src = key_src(bucket, nk);
     load_key_tile<D, CC>(tiles[0], src, nk);
   }
   while (true) {
-    // Items of this bucket inside [i0, i1) and their pairs.
-    const int it_lo = max(ws.item_off[bucket], i0);
-    const int it_hi = min(ws.item_off[bucket + 1], i1);
-    const int base = ws.bucket_off[bucket];
-    const int p_lo = base + (it_lo - ws.item_off[bucket]) * kPairsPerItem;
-    const int p_hi = min(base + (it_hi - ws.item_off[bucket]) * kPairsPerItem, ws.bucket_off[bucket + 1]);
-    // Next bucket with work inside the range: prefetch its tile.
-    int next = -1;
-    if (it_hi < i1) {
-      next = bucket + 1;
-      while (ws.item_off[next + 1] <= it_hi) ++next;  // skip buckets without items
+    const int p_lo = ws.bucket_off[bucket] + (item - ws.item_off[bucket]) * kPairsPerItem;
+    const int p_hi = min(p_lo + kPairsPerItem, ws.bucket_off[bucket + 1]);
+    const int next_item = item + gridDim.x;
+    const int next = next_item < total ? ws.item_bucket[next_item] : -1;
+    if (next >= 0 && next != bucket) {
       int nk;
       const bf16* src = key_src(next, nk);
       load_key_tile<D, CC>(tiles[buf ^ 1], src, nk);
@@ -381,7 +397,7 @@ __global__ void __launch_bounds__(kLeafThreads, 2)
     __syncthreads();
 
     const bf16* tile = tiles[buf];
-    const int64_t bh = bucket / M1;
+    const int64_t bh = bucket / bucket_span;
     const int64_t key0 = static_cast<int64_t>(bucket % M1) * CC;
     const int nkeys = static_cast<int>(min(static_cast<int64_t>(CC), a.N - key0));
     const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
@@ -471,8 +487,9 @@ __global__ void __launch_bounds__(kLeafThreads, 2)
     }
     if (next < 0) break;
     __syncthreads();  // every warp is done with tiles[buf] before it is refilled
+    if (next != bucket) buf ^= 1;
     bucket = next;
-    buf ^= 1;
+    item = next_item;
   }
 }
 
@@ -519,7 +536,7 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   carve(a, static_cast<char*>(ws_ptr), &ws);
   const int64_t rows = static_cast<int64_t>(a.B) * a.H_kv * a.N;
   const int M1 = static_cast<int>(level_size(a.N, a.C, 1));
-  const int nb = a.B * a.H_kv * M1;
+  const int nb = a.B * a.H_kv * ws.nwin * M1;
   cudaError_t e = cudaMemsetAsync(ws.count, 0, static_cast<size_t>(nb) * 4, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.fill, 0, static_cast<size_t>(nb) * 4, st);
   if (e != cudaSuccess) return e;
@@ -544,7 +561,9 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   count_launch();
   scatter_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(ws, rows, a.N, M1);
   count_launch();
-  const unsigned leaf_grid = static_cast<unsigned>(sm_count() * 2);
+  itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(ws, nb);
+  count_launch();
+  const unsigned leaf_grid = static_cast<unsigned>(sm_count() * 2);  // two 256-thread CTAs per SM
   e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
     constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
     if (a.C == 64)

@@ -80,6 +80,13 @@ int32_t pisa_version(void);
  * all entry points). Host-side counter; for accounting and tests. */
 uint64_t pisa_launch_count(void);
 
+/* Number of bounded device-side waits (on shared-memory copy barriers) that
+ * ran out of time on the current device since the library was loaded. Each
+ * such wait is abandoned after 2 s instead of hanging, so a non-zero count
+ * means some outputs are wrong. Diagnostic only: this call synchronises the
+ * device (it copies the counter to the host). Returns UINT64_MAX on error. */
+uint64_t pisa_device_faults(void);
+
 /*
  * Pyramid geometry (host only, pure integer arithmetic) — §Pyramid level
  * sizes: M_0 = N, M_1 = ceil(N / C), M_{l+1} = ceil(M_l / g) until M_L = 1.

@@ -95,3 +95,8 @@ def test_prefill_parity_full_size(name, rows):
     w = workloads.PREFILL[name]
     r = _run(w, rows)
     print(name, r)
+
+
+def test_no_device_wait_faults():
+    # Every bounded wait in the kernels completed (none was abandoned).
+    assert api.device_faults() == 0
