@@ -21,6 +21,7 @@
 #include "mma.cuh"
 #include "rowops.cuh"
 #include "select2.cuh"
+#include "tma.cuh"
 
 namespace pisa {
 
@@ -322,122 +323,158 @@ __global__ void __launch_bounds__(256) itemize_kernel(Ws ws, int nb) {
 }
 
 // ---------------------------------------------------------------- stage 2
-// Key tile layout in shared memory: row r (one key) holds D bf16 as D/8
-// 16-byte chunks; chunk ch is stored at position ch ^ 2 (r & 3). A 64-bit
-// fragment load is served per half-warp (rows gid = 0..3 or 4..7, two
-// chunks each); this swizzle puts those eight 8-byte reads in distinct banks.
-template <int D>
-__device__ inline uint2 key_frag(const bf16* tile, int r, int col) {
-  const int ch = col >> 3;
-  return *reinterpret_cast<const uint2*>(tile + r * D + ((ch ^ ((r & 3) << 1)) << 3) + (col & 7));
-}
-
-// Copies the C x D key tile of one leaf into shared memory (swizzled as
-// key_frag expects); rows past the sequence end are zero-filled.
-template <int D, int CC>
-__device__ inline void load_key_tile(bf16* tile, const bf16* __restrict__ ksrc, int nkeys) {
-  for (int x = threadIdx.x; x < CC * D / 8; x += blockDim.x) {
-    const int r = x / (D / 8), ch = x % (D / 8);
-    cp_async16(tile + r * D + ((ch ^ ((r & 3) << 1)) << 3), ksrc + (r < nkeys ? r * D + ch * 8 : 0), r < nkeys ? 16 : 0);
-  }
-  cp_async_commit();
-}
-
-// Stage 2. Each CTA owns a contiguous range of work items (64 pairs each,
-// ordered by bucket). Consecutive items of one bucket share the key tile in
-// shared memory; the next bucket's tile is prefetched (double buffer) while
-// the current one is scored. A warp scores one 16-row M tile at a time: the
-// 16 / G queries of a query tile (Q_tile = 4 queries x G heads is split into
-// passes of at most 16 rows), against all C keys of the tile.
+// Stage 2. Work items (64 pairs of one bucket) are walked grid-strided, so
+// that at any time all CTAs work on neighbouring buckets (the same query
+// window) and the window's queries stay in L2. Per item the leaf's C x d key
+// tile is brought into shared memory by bulk tensor copies (double buffered
+// across items, reused when the next item has the same bucket). Each warp
+// scores 16-row M tiles: the G heads of 16 / G queries (a query tile of
+// Q_tile = 4 queries x G heads is split into passes of 16 rows), whose rows
+// arrive as one 3-D tensor box per query (heads x d) in a per-warp double
+// buffer. Both MMA operands are read with ldmatrix from 128-byte swizzled
+// boxes. Per (query, head) row: LSE over the usable keys of the leaf; then
+// the sum over the G heads of each query.
 template <int D, int G, int CC>
 __global__ void __launch_bounds__(kLeafThreads, 2)
-    leaf_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, PrefillArgs a, Ws ws, int nb, int M1) {
-  constexpr int kNT = CC / 8;                 // 8-key N tiles per leaf
-  constexpr int kKS = D / 16;                 // 16-wide k steps
-  constexpr int kP = G >= 8 ? 2 : kQTile;     // queries per 16-row M tile
+    leaf_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk, PrefillArgs a,
+                Ws ws, int nb, int M1, unsigned long long* faults) {
+  constexpr int kNT = CC / 8;                  // 8-key N tiles per leaf
+  constexpr int kKS = D / 16;                  // 16-wide k steps
+  constexpr int kBoxes = D / 64;               // 64-column boxes per row
+  constexpr int kP = G >= 8 ? 2 : kQTile;      // queries per 16-row M tile
+  constexpr int kSlot = 1024;                  // one query's G rows of one box, 1 KB aligned
+  constexpr int kQStage = kP * kBoxes * kSlot;
+  constexpr int kKeyBytes = CC * D * 2;
+  constexpr int kWarps = kLeafThreads / 32;
   constexpr float kLog2e = 1.4426950408889634f;
-  __shared__ __align__(128) bf16 tiles[2][CC * D];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ uint64_t kbar[2];
+  __shared__ uint64_t qbar[kWarps][2];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
+  unsigned char* qring = smem + 2 * kKeyBytes + warp * 2 * kQStage;
   const bool causal = a.causal != 0;
   const float sl2 = a.scale * kLog2e;
+  if (threadIdx.x == 0) {
+    mbar_init(&kbar[0], 1);
+    mbar_init(&kbar[1], 1);
+  }
+  if (lane == 0) {
+    mbar_init(&qbar[warp][0], 1);
+    mbar_init(&qbar[warp][1], 1);
+  }
+  mbar_init_fence();
+  __syncthreads();
 
-  // Items are walked grid-strided, so that at any time all CTAs work on
-  // neighbouring buckets (the same query window) and the window's queries
-  // stay in L2. A tile is reused when the next item has the same bucket.
   const int total = ws.item_off[nb];
   int item = blockIdx.x;
   if (item >= total) return;
   const int64_t bucket_span = static_cast<int64_t>(ws.nwin) * M1;  // buckets per (b, kv head)
-  auto key_src = [&](int bk, int& nkeys) {
+  auto issue_key = [&](int bk, int bf) {  // thread 0 only
     const int64_t bhh = bk / bucket_span, leaf = bk % M1;
-    nkeys = static_cast<int>(min(static_cast<int64_t>(CC), a.N - leaf * CC));
-    return k + (bhh * a.N + leaf * CC) * D;
+    const int y = static_cast<int>(bhh * a.N + leaf * CC);
+    fence_proxy_async();
+    mbar_expect_tx(&kbar[bf], kKeyBytes);
+#pragma unroll
+    for (int x = 0; x < kBoxes; ++x) tma_load_2d(smem + bf * kKeyBytes + x * CC * 128, &tmk, 64 * x, y, &kbar[bf]);
   };
   int bucket = ws.item_bucket[item];
   int buf = 0;
-  {
-    int nk;
-    const bf16* src = key_src(bucket, nk);
-    load_key_tile<D, CC>(tiles[0], src, nk);
-  }
+  uint32_t kph = 0, kpend = 1;  // parity and pending-load bits per key buffer
+  if (threadIdx.x == 0) issue_key(bucket, 0);
+  int qst = 0;
+  uint32_t qph = 0;
+
   while (true) {
     const int p_lo = ws.bucket_off[bucket] + (item - ws.item_off[bucket]) * kPairsPerItem;
     const int p_hi = min(p_lo + kPairsPerItem, ws.bucket_off[bucket + 1]);
     const int next_item = item + gridDim.x;
     const int next = next_item < total ? ws.item_bucket[next_item] : -1;
     if (next >= 0 && next != bucket) {
-      int nk;
-      const bf16* src = key_src(next, nk);
-      load_key_tile<D, CC>(tiles[buf ^ 1], src, nk);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+      if (threadIdx.x == 0) issue_key(next, buf ^ 1);
+      kpend |= 1u << (buf ^ 1);
     }
-    __syncthreads();
-
-    const bf16* tile = tiles[buf];
+    if (kpend & (1u << buf)) {
+      mbar_wait(&kbar[buf], (kph >> buf) & 1u, faults);
+      kph ^= 1u << buf;
+      kpend &= ~(1u << buf);
+    }
+    const unsigned char* tile = smem + buf * kKeyBytes;
     const int64_t bh = bucket / bucket_span;
     const int64_t key0 = static_cast<int64_t>(bucket % M1) * CC;
     const int nkeys = static_cast<int>(min(static_cast<int64_t>(CC), a.N - key0));
     const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
-    const bf16* qbase = q + ((b * a.H_q + h * G) * a.N) * D + 4 * tig;
-    for (int u0 = p_lo + warp * kP; u0 < p_hi; u0 += nwarps * kP) {
-      const uint32_t pw = (lane < kP && u0 + lane < p_hi) ? ws.pairs[u0 + lane] : 0xffffffffu;
-      uint32_t a_reg[kKS][4];
+    const int zq = static_cast<int>(b * a.H_q + h * G);
+    const int nunits = (p_hi - p_lo + kP - 1) / kP;
+
+    // Queries of unit u into q stage st (lane 0 issues; one box per query per 64 columns).
+    auto issue_q = [&](int u, int st) {
+      if (lane == 0) {
+        const int pu = p_lo + u * kP;
+        const int nv = min(kP, p_hi - pu);
+        unsigned char* qs = qring + st * kQStage;
+        fence_proxy_async();
+        mbar_expect_tx(&qbar[warp][st], static_cast<uint32_t>(nv * G * D * 2));
+        for (int i = 0; i < nv; ++i) {
+          const int tq = static_cast<int>(ws.pairs[pu + i] >> 5);
+#pragma unroll
+          for (int x = 0; x < kBoxes; ++x)
+            tma_load_3d(qs + x * kP * kSlot + i * kSlot, &tmq, 64 * x, tq, zq, &qbar[warp][st]);
+        }
+      }
+    };
+    int u = warp;
+    if (u < nunits) issue_q(u, qst);
+    for (; u < nunits; u += kWarps) {
+      const int un = u + kWarps;
+      if (un < nunits) issue_q(un, qst ^ 1);
+      mbar_wait(&qbar[warp][qst], (qph >> qst) & 1u, faults);
+      qph ^= 1u << qst;
+      const unsigned char* qs = qring + qst * kQStage;
+
+      const int pu = p_lo + u * kP;
+      const uint32_t pw = (lane < kP && pu + lane < p_hi) ? ws.pairs[pu + lane] : 0xffffffffu;
       int nvk[2];
       bool ok[2];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int r = gid + 8 * half;
-        const int pi = r / G, hd = r % G;
+        const int pi = r / G;
         const uint32_t w = __shfl_sync(kFull, pw, pi < kP ? pi : 0);
         ok[half] = pi < kP && w != 0xffffffffu;
         const int64_t tq = ok[half] ? static_cast<int64_t>(w >> 5) : 0;
-        // usable keys of the tile for this query: [0, nvk)
         int64_t nv = nkeys;
         if (causal) nv = min(nv, tq - key0 + 1);
         nvk[half] = static_cast<int>(max(nv, static_cast<int64_t>(0)));
-        const bf16* qp = qbase + (static_cast<int64_t>(hd) * a.N + tq) * D;
-#pragma unroll
-        for (int ks = 0; ks < kKS; ++ks) {
-          uint2 uu = make_uint2(0u, 0u);
-          if (ok[half]) uu = *reinterpret_cast<const uint2*>(qp + 16 * ks);
-          a_reg[ks][half] = uu.x;
-          a_reg[ks][2 + half] = uu.y;
-        }
       }
+      // A (query rows) and B (keys) fragments via ldmatrix.
+      const int mat = lane >> 3, mr = lane & 7;
+      const int arow = mr + 8 * (mat & 1);                 // M-tile row this lane addresses
+      const int ap = arow / G < kP ? arow / G : 0, ag = arow % G;
+      const unsigned char* abase = qs + ap * kSlot + ag * 128;
       float acc[kNT][4];
 #pragma unroll
       for (int nt = 0; nt < kNT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
       for (int ks = 0; ks < kKS; ++ks) {
+        uint32_t af[4];
+        {
+          const int col = 16 * ks + 8 * (mat >> 1);
+          const int bx = col >> 6, c16 = (col & 63) >> 3;
+          ldsm_x4(af, abase + bx * kP * kSlot + ((c16 ^ (ag & 7)) << 4));
+        }
 #pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-          const uint2 bb = key_frag<D>(tile, 8 * nt + gid, 16 * ks + 4 * tig);
-          mma_bf16(acc[nt], a_reg[ks], bb.x, bb.y);
+        for (int nt = 0; nt < kNT; nt += 2) {
+          uint32_t bf[4];
+          const int krow = 8 * (nt + (mat >> 1)) + mr;
+          ldsm_x4(bf, tile + swz128<CC>(krow, 16 * ks + 8 * (mat & 1)));
+          mma_bf16(acc[nt], af, bf[0], bf[1]);
+          mma_bf16(acc[nt + 1], af, bf[2], bf[3]);
         }
       }
+      __syncwarp();  // the stage is refilled two units later
       // Per (query, head) row: LSE over the usable keys, in log2 units.
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -471,22 +508,23 @@ __global__ void __launch_bounds__(kLeafThreads, 2)
         }
         sum += __shfl_xor_sync(kFull, sum, 1);
         sum += __shfl_xor_sync(kFull, sum, 2);
-        float u = ok[half] ? mx * a.scale + logf(sum) : 0.f;
+        float uu = ok[half] ? mx * a.scale + logf(sum) : 0.f;
         // Sum over the G heads of each query: rows r .. r + G - 1 sit in
         // lanes that differ in the low log2(G) bits of gid.
 #pragma unroll
-        for (int o = 4; o < 4 * G; o <<= 1) u += __shfl_xor_sync(kFull, u, o);
+        for (int o = 4; o < 4 * G; o <<= 1) uu += __shfl_xor_sync(kFull, uu, o);
         const int r = gid + 8 * half;
         const int pi = r / G;
         const uint32_t w = __shfl_sync(kFull, pw, pi < kP ? pi : 0);
         if (tig == 0 && (gid % G) == 0 && ok[half]) {
           const int64_t orow = bh * a.N + static_cast<int64_t>(w >> 5);
-          ws.score[orow * 32 + (w & 31)] = u;
+          ws.score[orow * 32 + (w & 31)] = uu;
         }
       }
+      qst ^= 1;
     }
+    __syncthreads();  // every warp is done with the key tile (and its query stages)
     if (next < 0) break;
-    __syncthreads();  // every warp is done with tiles[buf] before it is refilled
     if (next != bucket) buf ^= 1;
     bucket = next;
     item = next_item;
@@ -563,19 +601,33 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   count_launch();
   itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(ws, nb);
   count_launch();
-  const unsigned leaf_grid = static_cast<unsigned>(sm_count() * 2);  // two 256-thread CTAs per SM
-  e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
-    constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
-    if (a.C == 64)
-      leaf_kernel<D, GG, 64><<<leaf_grid, kLeafThreads, 0, st>>>(static_cast<const bf16*>(q),
-                                                                  static_cast<const bf16*>(k), a, ws, nb, M1);
-    else
-      leaf_kernel<D, GG, 32><<<leaf_grid, kLeafThreads, 0, st>>>(static_cast<const bf16*>(q),
-                                                                  static_cast<const bf16*>(k), a, ws, nb, M1);
-    count_launch();
-    return cudaGetLastError();
-  });
-  if (e != cudaSuccess) return e;
+  {
+    CUtensorMap tmq, tmk;
+    const int G0 = a.H_q / a.H_kv;
+    e = make_tmap_bf16_3d(&tmq, q, a.d, a.N, static_cast<uint64_t>(a.B) * a.H_q, 1, G0);
+    if (e == cudaSuccess) e = make_tmap_bf16_2d(&tmk, k, a.d, static_cast<uint64_t>(a.B) * a.H_kv * a.N, a.C);
+    if (e != cudaSuccess) return e;
+    unsigned long long* faults = wait_fault_counter();
+    e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
+      constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
+      constexpr int kP = GG >= 8 ? 2 : kQTile;
+      const size_t qstage = static_cast<size_t>(kP) * (D / 64) * 1024;
+      auto launch = [&](auto kern, int CC) -> cudaError_t {
+        const size_t smem = 2 * static_cast<size_t>(CC) * D * 2 + (kLeafThreads / 32) * 2 * qstage + 1024;
+        cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e2 != cudaSuccess) return e2;
+        int per_sm = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLeafThreads, smem) != cudaSuccess ||
+            per_sm < 1)
+          per_sm = 1;
+        kern<<<static_cast<unsigned>(sm_count() * per_sm), kLeafThreads, smem, st>>>(tmq, tmk, a, ws, nb, M1, faults);
+        count_launch();
+        return cudaGetLastError();
+      };
+      return a.C == 64 ? launch(leaf_kernel<D, GG, 64>, 64) : launch(leaf_kernel<D, GG, 32>, 32);
+    });
+    if (e != cudaSuccess) return e;
+  }
   final_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(a, ws, sel, sel_score, rows);
   count_launch();
   return cudaGetLastError();

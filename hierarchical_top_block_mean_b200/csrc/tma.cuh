@@ -19,6 +19,11 @@ namespace pisa {
 // rows read as zero.
 cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows);
 
+// 3-D bf16 tensor map over [d2][d1][d0] (d0 innermost) with a box of
+// 64 x box1 x box2 elements and 128-byte swizzle.
+cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                              uint32_t box1, uint32_t box2);
+
 // Device address of the fault counter (bounded waits that ran out) on the
 // current device; kernels that wait take it as an argument.
 unsigned long long* wait_fault_counter();
@@ -65,6 +70,25 @@ __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long l
     }
   }
   return true;
+}
+
+__device__ inline void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ inline void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ inline void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
 }
 
 // Orders this thread's earlier generic-proxy accesses to shared memory
