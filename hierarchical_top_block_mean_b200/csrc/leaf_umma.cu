@@ -1,0 +1,390 @@
+// Stage-2 leaf scorer on the fifth-generation tensor cores (tcgen05) for
+// groups of G_Q = 8 query heads, d = 128, C = 64 (the paper's kernel
+// design, §Kernels: a d x C key tile reused across a (Q_tile G_Q) x d query
+// tile).
+//
+// One CTA per SM runs a warp-specialised pipeline over the stage-2 work
+// items (64 (query, leaf) pairs of one bucket, walked grid-strided so that
+// all SMs share the current query window in L2):
+//   warps 4-5 (loads): per tile of 16 queries, their 8 head rows
+//     (16 x 8 = 128 rows) gathered with 16-byte cp.async straight into the
+//     swizzled operand layout of a ring of query stages, running ahead of the
+//     MMAs (many small bulk copies cost more than one per 2 KB row group);
+//   warp 6, one lane (MMA): per item, the leaf's 64 x 128 key tile by bulk
+//     tensor copy, issued one item ahead into a double buffer; per tile, eight
+//     tcgen05.mma (M = 128 query-head
+//     rows, N = 64 keys, K = 16 each) into a ring of TMEM accumulators,
+//     then tcgen05.commit to release the query stage (and, after an item's
+//     last tile, the key tile) and to publish the accumulator;
+//   warps 0-3 (epilogue): each thread owns one TMEM lane = one (query, head)
+//     row, loads its 64 key scores with tcgen05.ld, takes the LSE over the
+//     usable keys in registers, sums the 8 heads of its query with three
+//     shuffles, and one lane per query stores the leaf score.
+// Operands sit in shared memory as 128-byte-swizzled K-major tiles (rows of
+// 64 bf16, 8-row groups 1 KB apart), which is both the bulk-copy layout and
+// the MMA descriptor layout. Every mbarrier wait is bounded in time; the
+// TMEM allocation is always released before exit.
+#include "dispatch.cuh"
+#include "select2_ws.cuh"
+#include "tma.cuh"
+
+namespace pisa {
+
+namespace {
+
+constexpr int kUmmaThreads = 224;          // warps 0-3 epilogue, warps 4-5 loads, warp 6 MMA issue
+constexpr int kLoaders = 64;               // threads of warps 4-5
+constexpr int kTilePairs = 16;             // queries per MMA tile (x 8 heads = 128 rows)
+constexpr int kQStages = 4;
+constexpr int kQStageBytes = kTilePairs * 8 * 128 * 2;  // 16 queries x 8 heads x 256 B = 32 KB (two 64-col halves)
+constexpr int kKeyBytes = 64 * 128 * 2;                 // 16 KB (two 64-col halves)
+constexpr int kAccCols = 64;                            // fp32 columns per accumulator (N = 64 keys)
+constexpr int kAccStages = 4;                           // TMEM accumulator buffers
+constexpr uint32_t kTmemCols = kAccStages * kAccCols;
+
+__device__ inline void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+}
+__device__ inline void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ inline void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ inline void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ inline void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+// D[tmem] (+)= A . B^T with A [M x K] and B [N x K] K-major in shared memory.
+__device__ inline void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Arrives on bar once every tcgen05.mma issued so far by this thread is complete.
+__device__ inline void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+}
+__device__ inline void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+// 16-byte cp.async global -> shared.
+__device__ inline void cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ inline void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ inline void cp_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+__device__ inline void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), descriptor version 1.
+__device__ inline uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1) << 16;              // leading byte offset (unused for swizzled K-major)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;      // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;              // version
+  d |= static_cast<uint64_t>(2) << 61;              // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, both
+// K-major, N = 64, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+
+struct Cursor2 {
+  int item, bucket, p_lo, p_hi, ntiles;
+};
+
+__global__ void __launch_bounds__(kUmmaThreads, 1)
+    leaf_umma_kernel(const bf16* __restrict__ q, const __grid_constant__ CUtensorMap tmk, PrefillArgs a, Ws ws,
+                     int nb, int M1, unsigned long long* faults) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ uint64_t kfull[2], kempty[2], qfull[kQStages], qempty[kQStages], accfull[kAccStages], accempty[kAccStages];
+  __shared__ uint32_t tmem_base_sh;
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* kbuf = smem;                       // [2][kKeyBytes]
+  unsigned char* qbuf = smem + 2 * kKeyBytes;       // [kQStages][kQStageBytes]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kfull[i], 1);
+      mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < kAccStages; ++i) {
+      mbar_init(&accfull[i], 1);
+      mbar_init(&accempty[i], 4);
+    }
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&qfull[i], kLoaders);
+      mbar_init(&qempty[i], 1);
+    }
+    mbar_init_fence();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  const int total = ws.item_off[nb];
+  const int64_t bucket_span = static_cast<int64_t>(ws.nwin) * M1;
+  const bool causal = a.causal != 0;
+  // Work-item records are loaded one item ahead (one 16-byte load each).
+  auto info = [&](int item) { return item < total ? ws.item_info[item] : make_int4(0, 0, 0, 0); };
+  auto cursor = [&](int item, int4 inf) {
+    Cursor2 c;
+    c.item = item;
+    c.bucket = inf.x;
+    c.p_lo = inf.y;
+    c.p_hi = inf.z;
+    c.ntiles = (c.p_hi - c.p_lo + kTilePairs - 1) / kTilePairs;
+    return c;
+  };
+
+  if (warp == 4 || warp == 5) {
+    // ---------------------------------------------------------- loads
+    const int lw = warp - 4;                      // loader warp 0..1
+    const int jcol = lane & 15;                   // 16-byte column of a 256-byte query row
+    const int g0 = 2 * lw + (lane >> 4);          // head rows g0 and g0 + 4
+    const int64_t head_stride = static_cast<int64_t>(a.N) * 128;
+    int nq = 0;                        // uses of the query ring so far
+    int pend[3] = {0, 0, 0}, np_head = 0, npend = 0;  // filled stages not yet published (FIFO)
+    int4 inf = info(blockIdx.x);
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+      const Cursor2 c = cursor(item, inf);
+      inf = info(item + gridDim.x);
+      const int64_t bh = c.bucket / bucket_span;
+      const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
+      const bf16* qg = q + (b * a.H_q + h * 8) * static_cast<int64_t>(a.N) * 128;  // head 0 of the group
+      const bf16* qrow0 = qg + g0 * head_stride + jcol * 8;                        // this thread's column of head g0
+      for (int tl = 0; tl < c.ntiles; ++tl) {
+        const int qs = nq % kQStages;
+        const int p0 = c.p_lo + tl * kTilePairs;
+        const int np = min(kTilePairs, c.p_hi - p0);
+        // Loader thread (warp lw, lane l): 16-byte column j = l & 15 of head
+        // rows g0 and g0 + 4 (g0 = 2 lw + (l >> 4)) of every query of the tile,
+        // so each copy instruction moves two whole 256-byte rows. The tile's
+        // query positions are read once per warp and shared by shuffle.
+        const int tw = lane < np ? static_cast<int>(ws.pairs[p0 + lane] >> 5) : 0;
+        mbar_wait(&qempty[qs], ((nq / kQStages) & 1) ^ 1, faults);
+        const uint32_t qd = smem_u32(qbuf + qs * kQStageBytes);
+        const uint32_t d0 = qd + (jcol >> 3) * (kQStageBytes / 2) + g0 * 128 + (((jcol & 7) ^ g0) << 4);
+        const uint32_t d1 = qd + (jcol >> 3) * (kQStageBytes / 2) + (g0 + 4) * 128 + (((jcol & 7) ^ (g0 + 4)) << 4);
+        for (int i = 0; i < np; ++i) {
+          const int tq = __shfl_sync(kFull, tw, i);
+          const bf16* src = qrow0 + static_cast<int64_t>(tq) * 128;
+          cp16(d0 + i * 1024, src);
+          cp16(d1 + i * 1024, src + 4 * head_stride);
+        }
+        cp_commit();
+        // Publish the stage filled two tiles ago: its copies have landed
+        // (at most two newer groups pending), and the proxy fence makes these
+        // generic-proxy writes visible to the tensor cores' async-proxy reads.
+        pend[(np_head + npend) % 3] = qs;
+        ++npend;
+        if (npend > 2) {
+          cp_wait<2>();
+          fence_proxy_async();
+          mbar_arrive(&qfull[pend[np_head]]);
+          np_head = (np_head + 1) % 3;
+          --npend;
+        }
+        ++nq;
+      }
+    }
+    cp_wait<0>();
+    fence_proxy_async();
+    for (; npend > 0; --npend) {
+      mbar_arrive(&qfull[pend[np_head]]);
+      np_head = (np_head + 1) % 3;
+    }
+  } else if (warp == 6) {
+    // ---------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      int nk = 0, nq = 0, na = 0;
+      // Key tiles are loaded by this thread one item ahead; a key buffer is
+      // refilled only after this thread's own commit of its last MMAs.
+      auto load_key = [&](int4 ki, int n) {
+        const int kbn = n & 1;
+        mbar_wait(&kempty[kbn], ((n >> 1) & 1) ^ 1, faults);
+        const int64_t bhk = ki.x / bucket_span, leafk = ki.x % M1;
+        const int ky = static_cast<int>(bhk * a.N + leafk * 64);
+        fence_proxy_async();
+        mbar_expect_tx(&kfull[kbn], kKeyBytes);
+        tma_load_2d(kbuf + kbn * kKeyBytes, &tmk, 0, ky, &kfull[kbn]);
+        tma_load_2d(kbuf + kbn * kKeyBytes + 64 * 128, &tmk, 64, ky, &kfull[kbn]);
+      };
+      int4 inf = info(blockIdx.x);
+      if (blockIdx.x < total) load_key(inf, 0);
+      for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const Cursor2 c = cursor(item, inf);
+        inf = info(item + gridDim.x);
+        if (item + gridDim.x < total) load_key(inf, nk + 1);
+        const int kb = nk & 1;
+        mbar_wait(&kfull[kb], (nk >> 1) & 1, faults);
+        const uint32_t ka = smem_u32(kbuf + kb * kKeyBytes);
+        for (int tl = 0; tl < c.ntiles; ++tl) {
+          const int qs = nq % kQStages;
+          mbar_wait(&qfull[qs], (nq / kQStages) & 1, faults);
+          const int as = na % kAccStages;
+          mbar_wait(&accempty[as], ((na / kAccStages) & 1) ^ 1, faults);
+          tc_fence_after();
+          const uint32_t qa = smem_u32(qbuf + qs * kQStageBytes);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * (kQStageBytes / 2) + (ks & 3) * 32;
+            const uint32_t koff = (ks >> 2) * (64 * 128) + (ks & 3) * 32;
+            umma_bf16(tmem + as * kAccCols, sw128_desc(qa + off), sw128_desc(ka + koff), kIdesc, ks > 0);
+          }
+          umma_commit(&qempty[qs]);
+          umma_commit(&accfull[as]);
+          ++nq;
+          ++na;
+        }
+        umma_commit(&kempty[kb]);
+        ++nk;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    // Tiles are walked as one stream; each row's (query, slot) word is
+    // loaded one tile ahead so its latency hides behind the current tile.
+    const float sl2 = a.scale * 1.4426950408889634f;
+    const int row = 32 * warp + lane;  // TMEM lane = (query, head) row of the tile
+    int na = 0;
+    int item = blockIdx.x;
+    Cursor2 c = cursor(item, info(item));
+    int4 inf_next = info(item + gridDim.x);
+    int tl = 0;
+    auto pair_word = [&](const Cursor2& cc, int t) -> uint32_t {
+      const int p = cc.p_lo + t * kTilePairs + row / 8;
+      return p < cc.p_hi ? ws.pairs[p] : 0xffffffffu;
+    };
+    uint32_t w_next = item < total ? pair_word(c, 0) : 0xffffffffu;
+    while (item < total) {
+      const uint32_t w = w_next;
+      const bool ok = w != 0xffffffffu;
+      const int64_t bh = c.bucket / bucket_span;
+      const int64_t key0 = static_cast<int64_t>(c.bucket % M1) * 64;
+      const int nkeys = static_cast<int>(min(static_cast<int64_t>(64), a.N - key0));
+      // Advance the stream and prefetch the next tile's word.
+      Cursor2 cn = c;
+      int tln = tl + 1, itemn = item;
+      if (tln >= c.ntiles) {
+        itemn = item + gridDim.x;
+        tln = 0;
+        if (itemn < total) {
+          cn = cursor(itemn, inf_next);
+          inf_next = info(itemn + gridDim.x);
+        }
+      }
+      w_next = itemn < total ? pair_word(cn, tln) : 0xffffffffu;
+
+      const int as = na % kAccStages;
+      mbar_wait(&accfull[as], (na / kAccStages) & 1, faults);
+      tc_fence_after();
+      uint32_t v[64];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + as * kAccCols;
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+        tmem_ld32(taddr, lo);
+        tmem_ld32(taddr + 32, hi);
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[as]);
+      ++na;
+      int nv = nkeys;
+      if (causal && ok) nv = static_cast<int>(min(static_cast<int64_t>(nv), static_cast<int64_t>(w >> 5) - key0 + 1));
+      float mx = -INFINITY;
+      if (nv >= 64) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          if (j < nv) mx = fmaxf(mx, __uint_as_float(v[j]));
+      }
+      const float mxs = mx * sl2;
+      // Four partial sums shorten the dependent add chain.
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (nv >= 64) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) s4[j & 3] += exp2f(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          if (j < nv) s4[j & 3] += exp2f(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+      }
+      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      float u = ok ? mx * a.scale + logf(sum) : 0.f;
+      u += __shfl_xor_sync(kFull, u, 1);
+      u += __shfl_xor_sync(kFull, u, 2);
+      u += __shfl_xor_sync(kFull, u, 4);
+      if (ok && (row & 7) == 0) {
+        const int64_t orow = bh * a.N + static_cast<int64_t>(w >> 5);
+        ws.score[orow * 32 + (w & 31)] = u;
+      }
+      c = cn;
+      tl = tln;
+      item = itemn;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+int sm_count_umma() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+bool leaf_umma_supported(const PrefillArgs& a) {
+  return a.dtype == PISA_DTYPE_BF16 && a.d == 128 && a.C == 64 && a.H_q == 8 * a.H_kv;
+}
+
+cudaError_t launch_leaf_umma(const PrefillArgs& a, const void* q, const void* k, const Ws& ws, int nb, int M1,
+                             cudaStream_t st) {
+  CUtensorMap tmk;
+  cudaError_t e = make_tmap_bf16_2d(&tmk, k, a.d, static_cast<uint64_t>(a.B) * a.H_kv * a.N, 64);
+  if (e != cudaSuccess) return e;
+  const size_t smem = 2 * static_cast<size_t>(kKeyBytes) + kQStages * static_cast<size_t>(kQStageBytes) + 1024;
+  e = cudaFuncSetAttribute(leaf_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  leaf_umma_kernel<<<static_cast<unsigned>(sm_count_umma()), kUmmaThreads, smem, st>>>(
+      static_cast<const bf16*>(q), tmk, a, ws, nb, M1, wait_fault_counter());
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace pisa

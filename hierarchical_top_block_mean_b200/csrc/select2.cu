@@ -21,6 +21,7 @@
 #include "mma.cuh"
 #include "rowops.cuh"
 #include "select2.cuh"
+#include "select2_ws.cuh"
 #include "tma.cuh"
 
 namespace pisa {
@@ -31,22 +32,6 @@ constexpr int kRouterWarps = 4;
 constexpr int kPairsPerItem = 64;  // stage-2 work item: 16 query tiles of Q_tile = 4 pairs
 constexpr int kQTile = 4;
 constexpr int kLeafThreads = 256;
-
-// Workspace sections (all 256-byte aligned).
-struct Ws {
-  int32_t* cand;        // [rows][32] candidate leaves per row after stage 1 (-1 padded)
-  int32_t* ncand;       // [rows] candidates per row; -1 when stage 1 already wrote sel
-  float* score;         // [rows][32] leaf score of each candidate slot
-  int32_t* count;       // [buckets] pairs per (b, kv head, leaf)
-  int32_t* fill;        // [buckets] scatter cursors
-  int32_t* bucket_off;  // [buckets + 1] exclusive scan of count
-  int32_t* item_off;    // [buckets + 1] exclusive scan of ceil(count / kPairsPerItem)
-  uint32_t* pairs;      // [rows * 32] (t << 5 | slot), grouped by bucket
-  uint4* planes;        // [B*H_kv][R][D/4] pyramid rows as bf16 hi/lo: {hi x4, lo x4} per 4 elements
-  int32_t* item_bucket; // [items] bucket of each stage-2 work item
-  int win_shift;        // queries are bucketed by window t >> win_shift
-  int nwin;             // windows per (b, kv head)
-};
 
 // Query window of the stage-2 buckets: about 32 MB of one kv head's queries
 // (W x G_Q x d x 2 bytes), so that a window's queries stay L2-resident while
@@ -82,6 +67,7 @@ size_t carve(const PrefillArgs& a, char* base, Ws* w) {
   x.pairs = reinterpret_cast<uint32_t*>(take(rows * 32 * 4));
   x.planes = reinterpret_cast<uint4*>(take(static_cast<size_t>(a.B) * a.H_kv * make_layout(a.N, a.C).R * a.d * 4));
   x.item_bucket = reinterpret_cast<int32_t*>(take((rows * 32 / kPairsPerItem + nb + 1) * 4));
+  x.item_info = reinterpret_cast<int4*>(take((rows * 32 / kPairsPerItem + nb + 1) * 16));
   x.win_shift = sh;
   x.nwin = nwin;
   if (w) *w = x;
@@ -315,11 +301,17 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ws ws, int64_t rows, int N
   ws.pairs[ws.bucket_off[bucket] + pos] = (static_cast<uint32_t>(t) << 5) | static_cast<uint32_t>(slot);
 }
 
-// Item -> bucket map: one thread per bucket writes its items' entries.
+// Item -> (bucket, pair range) map: one thread per bucket writes its items' entries.
 __global__ void __launch_bounds__(256) itemize_kernel(Ws ws, int nb) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= nb) return;
-  for (int i = ws.item_off[b]; i < ws.item_off[b + 1]; ++i) ws.item_bucket[i] = b;
+  const int i0 = ws.item_off[b], i1 = ws.item_off[b + 1];
+  const int p0 = ws.bucket_off[b], p1 = ws.bucket_off[b + 1];
+  for (int i = i0; i < i1; ++i) {
+    ws.item_bucket[i] = b;
+    const int lo = p0 + (i - i0) * kPairsPerItem;
+    ws.item_info[i] = make_int4(b, lo, min(lo + kPairsPerItem, p1), 0);
+  }
 }
 
 // ---------------------------------------------------------------- stage 2
@@ -601,7 +593,9 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   count_launch();
   itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(ws, nb);
   count_launch();
-  {
+  if (leaf_umma_supported(a)) {
+    if ((e = launch_leaf_umma(a, q, k, ws, nb, M1, st)) != cudaSuccess) return e;
+  } else {
     CUtensorMap tmq, tmk;
     const int G0 = a.H_q / a.H_kv;
     e = make_tmap_bf16_3d(&tmq, q, a.d, a.N, static_cast<uint64_t>(a.B) * a.H_q, 1, G0);
