@@ -6,11 +6,11 @@
 // One CTA per SM runs a warp-specialised pipeline over the stage-2 work
 // items (64 (query, leaf) pairs of one bucket, walked grid-strided so that
 // all SMs share the current query window in L2):
-//   warps 4-5 (loads): per tile of 16 queries, their 8 head rows
+//   warps 4-7 (loads): per tile of 16 queries, their 8 head rows
 //     (16 x 8 = 128 rows) gathered with 16-byte cp.async straight into the
 //     swizzled operand layout of a ring of query stages, running ahead of the
 //     MMAs (many small bulk copies cost more than one per 2 KB row group);
-//   warp 6, one lane (MMA): per item, the leaf's 64 x 128 key tile by bulk
+//   warp 8, one lane (MMA): per item, the leaf's 64 x 128 key tile by bulk
 //     tensor copy, issued one item ahead into a double buffer; per tile, eight
 //     tcgen05.mma (M = 128 query-head
 //     rows, N = 64 keys, K = 16 each) into a ring of TMEM accumulators,
@@ -32,10 +32,12 @@ namespace pisa {
 
 namespace {
 
-constexpr int kUmmaThreads = 224;          // warps 0-3 epilogue, warps 4-5 loads, warp 6 MMA issue
-constexpr int kLoaders = 64;               // threads of warps 4-5
+constexpr int kLoadWarps = 4;              // warps 4-7 gather the query rows
+constexpr int kMmaWarp = 4 + kLoadWarps;   // warp 8 issues the MMAs
+constexpr int kUmmaThreads = 32 * (kMmaWarp + 1);
+constexpr int kLoaders = 32 * kLoadWarps;
 constexpr int kTilePairs = 16;             // queries per MMA tile (x 8 heads = 128 rows)
-constexpr int kQStages = 4;
+constexpr int kQStages = 5;
 constexpr int kQStageBytes = kTilePairs * 8 * 128 * 2;  // 16 queries x 8 heads x 256 B = 32 KB (two 64-col halves)
 constexpr int kKeyBytes = 64 * 128 * 2;                 // 16 KB (two 64-col halves)
 constexpr int kAccCols = 64;                            // fp32 columns per accumulator (N = 64 keys)
@@ -157,11 +159,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     return c;
   };
 
-  if (warp == 4 || warp == 5) {
+  if (warp >= 4 && warp < kMmaWarp) {
     // ---------------------------------------------------------- loads
-    const int lw = warp - 4;                      // loader warp 0..1
+    const int lw = warp - 4;                      // loader warp 0..kLoadWarps-1
     const int jcol = lane & 15;                   // 16-byte column of a 256-byte query row
-    const int g0 = 2 * lw + (lane >> 4);          // head rows g0 and g0 + 4
+    const int g0 = 2 * lw + (lane >> 4);          // head row g0 (and g0 + 4 with two loader warps)
     const int64_t head_stride = static_cast<int64_t>(a.N) * 128;
     int nq = 0;                        // uses of the query ring so far
     int pend[3] = {0, 0, 0}, np_head = 0, npend = 0;  // filled stages not yet published (FIFO)
@@ -178,19 +180,22 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         const int p0 = c.p_lo + tl * kTilePairs;
         const int np = min(kTilePairs, c.p_hi - p0);
         // Loader thread (warp lw, lane l): 16-byte column j = l & 15 of head
-        // rows g0 and g0 + 4 (g0 = 2 lw + (l >> 4)) of every query of the tile,
+        // row g0 = 2 lw + (l >> 4) (and g0 + 4 with two loader warps) of every query of the tile,
         // so each copy instruction moves two whole 256-byte rows. The tile's
         // query positions are read once per warp and shared by shuffle.
         const int tw = lane < np ? static_cast<int>(ws.pairs[p0 + lane] >> 5) : 0;
         mbar_wait(&qempty[qs], ((nq / kQStages) & 1) ^ 1, faults);
         const uint32_t qd = smem_u32(qbuf + qs * kQStageBytes);
         const uint32_t d0 = qd + (jcol >> 3) * (kQStageBytes / 2) + g0 * 128 + (((jcol & 7) ^ g0) << 4);
-        const uint32_t d1 = qd + (jcol >> 3) * (kQStageBytes / 2) + (g0 + 4) * 128 + (((jcol & 7) ^ (g0 + 4)) << 4);
         for (int i = 0; i < np; ++i) {
           const int tq = __shfl_sync(kFull, tw, i);
           const bf16* src = qrow0 + static_cast<int64_t>(tq) * 128;
           cp16(d0 + i * 1024, src);
-          cp16(d1 + i * 1024, src + 4 * head_stride);
+          if (kLoadWarps == 2) {
+            const uint32_t d1 =
+                qd + (jcol >> 3) * (kQStageBytes / 2) + (g0 + 4) * 128 + (((jcol & 7) ^ (g0 + 4)) << 4);
+            cp16(d1 + i * 1024, src + 4 * head_stride);
+          }
         }
         cp_commit();
         // Publish the stage filled two tiles ago: its copies have landed
@@ -214,7 +219,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       mbar_arrive(&qfull[pend[np_head]]);
       np_head = (np_head + 1) % 3;
     }
-  } else if (warp == 6) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
       int nk = 0, nq = 0, na = 0;
