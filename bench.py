@@ -157,17 +157,20 @@ def pyramid_bytes(w) -> float:
 
 def measured_traffic(workload: str, kernel: str):
     """DRAM bytes per launch of `kernel` recorded by an ncu capture in
-    profiles/traffic.json, or None when absent or when the kernel's source
-    has changed since the capture (the recorded sha256 no longer matches)."""
+    profiles/traffic.json, or None when absent or when any of the kernel's
+    source files has changed since the capture (the recorded sha256 of the
+    concatenated sources no longer matches)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[workload][kernel]
-        src = os.path.join(ROOT, rec["source"])
-        with open(src, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
-                return None
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["sha256"]:
+            return None
         return rec["dram_read_bytes"] + rec["dram_write_bytes"]
     except (OSError, KeyError, ValueError):
         return None
