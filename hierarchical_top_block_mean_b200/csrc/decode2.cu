@@ -36,6 +36,12 @@ namespace {
 constexpr int kDecWarps = 8;
 constexpr int kModeAppend = 1, kModeSelect = 2, kModeAttend = 4;
 
+// Asks the memory system to bring `bytes` (a multiple of 16) starting at p
+// into L2, without waiting; later loads of the range then hit L2.
+__device__ inline void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Raw-key LSE of one leaf block summed over the G heads, by one warp
 // (S^T = K Q^T on tensor cores; keys at or beyond n are excluded).
 template <int D, int CC, int G>
@@ -92,7 +98,7 @@ __device__ inline float leaf_lse(const bf16* __restrict__ kh, int64_t key0, int6
 }
 
 template <int D, int CC, int G>
-__global__ void __launch_bounds__(kDecWarps * 32)
+__global__ void __launch_bounds__(kDecWarps * 32, 2)
     decode_kernel(DecodeArgs a, Layout lay, int mode, const bf16* __restrict__ q_new, const bf16* __restrict__ k_new,
                   const bf16* __restrict__ v_new, bf16* __restrict__ kc, bf16* __restrict__ vc,
                   float* __restrict__ pyr, int32_t* __restrict__ len, int32_t* __restrict__ sel,
@@ -236,6 +242,13 @@ __global__ void __launch_bounds__(kDecWarps * 32)
               if (tig == 0 && have) score[8 * m + gid] = u;
             }
           } else {
+            // All candidate leaves' key tiles are requested into L2 at once, so
+            // their DRAM fetches overlap instead of following one another.
+            if (threadIdx.x < nc) {
+              const int64_t k0 = static_cast<int64_t>(cand[threadIdx.x]) * CC;
+              const int64_t nk = (k0 + CC <= nn ? CC : nn - k0);
+              prefetch_l2(kh + k0 * D, static_cast<uint32_t>(nk * D * 2));
+            }
             for (int x = warp; x < nc; x += kDecWarps) {
               const float u = leaf_lse<D, CC, G>(kh, static_cast<int64_t>(cand[x]) * CC, nn, qb, a.scale);
               if (lane == 0) score[x] = u;
@@ -272,6 +285,15 @@ __global__ void __launch_bounds__(kDecWarps * 32)
   __syncthreads();
 
   if (mode & kModeAttend) {
+    // The selected blocks' K and V rows are requested into L2 together.
+    if (threadIdx.x < 2 * K) {
+      const int bsel = blk[threadIdx.x >> 1];
+      if (bsel >= 0) {
+        const int64_t k0 = static_cast<int64_t>(bsel) * CC;
+        const int64_t nk = (k0 + CC <= nn ? CC : nn - k0);
+        prefetch_l2(((threadIdx.x & 1) ? vh : kh) + k0 * D, static_cast<uint32_t>(nk * D * 2));
+      }
+    }
     MmaAttend<D, CC, G> at;
     at.m[0] = at.m[1] = -INFINITY;
     at.l[0] = at.l[1] = 0.f;
