@@ -55,11 +55,12 @@ SIGNATURES = {
     "pisa_sparse_attn_fwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p]),
     "pisa_select_noalloc": (_i32, [_PC, _p, _p, _p, _p, _p, _p]),
     "pisa_decode_pyramid_rows": (_i64, [_PD]),
+    "pisa_decode_workspace_bytes": (_i64, [_PD]),
     "pisa_decode_init": (_i32, [_PD, _p, _p, _p, _p]),
     "pisa_decode_append": (_i32, [_PD, _p, _p, _p, _p, _p, _p, _p, _p]),
     "pisa_decode_select": (_i32, [_PD, _p, _p, _p, _p, _p, _p]),
-    "pisa_decode_attn": (_i32, [_PD, _p, _p, _p, _p, _p, _p, _p, _p]),
-    "pisa_decode_step": (_i32, [_PD, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "pisa_decode_attn": (_i32, [_PD, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "pisa_decode_step": (_i32, [_PD, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
 }
 
 _lock = threading.Lock()

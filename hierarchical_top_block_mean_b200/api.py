@@ -198,7 +198,8 @@ def prefill(q, k, v, *, C: int, K: int, causal: bool, scale: float = 0.0):
 
 class DecodeState:
     """Caller-side decode state for S sequences of capacity cap: KV caches,
-    the cached mean pyramid, per-sequence lengths and a device status word."""
+    the cached mean pyramid, per-sequence lengths, a device status word and
+    the decode workspace."""
 
     def __init__(self, *, S: int, cap: int, H_q: int, H_kv: int, d: int, C: int, K: int,
                  dtype=torch.bfloat16, scale: float = 0.0, device="cuda", k_cache=None, v_cache=None, lens=None):
@@ -221,6 +222,8 @@ class DecodeState:
         self.sel = torch.empty((S, H_kv, K), dtype=torch.int32, device=dev)
         self.out = torch.empty((S, H_q, d), dtype=dtype, device=dev)
         self.lse = torch.empty((S, H_q), dtype=torch.float32, device=dev)
+        ws = int(_lib.lib().pisa_decode_workspace_bytes(ctypes.byref(self.cfg)))
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
 
     def init(self):
         """Builds each sequence's pyramid over its first len[s] cached tokens."""
@@ -239,14 +242,14 @@ class DecodeState:
     def attend(self, q_new, sel=None):
         s = self.sel if sel is None else sel
         _lib.call("pisa_decode_attn", ctypes.byref(self.cfg), _p(q_new), _p(self.k_cache), _p(self.v_cache),
-                  _p(self.len), _p(s), _p(self.out), _p(self.lse), _stream(self.pyr))
+                  _p(self.len), _p(s), _p(self.out), _p(self.lse), _p(self.workspace), _stream(self.pyr))
         return self.out
 
     def step(self, q_new, k_new, v_new, keep_sel: bool = True):
         """Append + select + attend for every sequence."""
         _lib.call("pisa_decode_step", ctypes.byref(self.cfg), _p(q_new), _p(k_new), _p(v_new), _p(self.k_cache),
                   _p(self.v_cache), _p(self.pyr), _p(self.len), _p(self.sel) if keep_sel else None, _p(self.out),
-                  _p(self.lse), _p(self.status), _stream(self.pyr))
+                  _p(self.lse), _p(self.status), _p(self.workspace), _stream(self.pyr))
         return self.out
 
     def level_offsets(self):

@@ -170,6 +170,12 @@ int64_t pisa_decode_pyramid_rows(const pisa_decode_config* cfg) {
   return make_layout(cfg->cap, cfg->C).R;
 }
 
+int64_t pisa_decode_workspace_bytes(const pisa_decode_config* cfg) {
+  if (check_dcfg(cfg) != PISA_OK) return 0;
+  const DecodeArgs a = dargs_of(cfg);
+  return decode_fused_supported(a) ? decode_logit_floats(a) * 4 : 0;
+}
+
 pisa_status pisa_decode_init(const pisa_decode_config* cfg, const void* k_cache, float* pyr, const int32_t* len,
                              void* stream) {
   pisa_status s = check_dcfg(cfg);
@@ -190,7 +196,7 @@ pisa_status pisa_decode_append(const pisa_decode_config* cfg, const void* k_new,
   const DecodeArgs a = dargs_of(cfg);
   if (decode_fused_supported(a))
     return from_cuda(launch_decode_fused(a, lay, 1, nullptr, k_new, v_new, k_cache, v_cache, pyr, len, nullptr, nullptr,
-                                         nullptr, status, as_stream(stream)));
+                                         nullptr, status, nullptr, as_stream(stream)));
   return from_cuda(launch_decode_append(a, lay, k_new, v_new, k_cache, v_cache, pyr, len, status, as_stream(stream)));
 }
 
@@ -205,7 +211,7 @@ pisa_status pisa_decode_select(const pisa_decode_config* cfg, const void* q_new,
   if (decode_fused_supported(a))
     return from_cuda(launch_decode_fused(a, lay, 2, q_new, nullptr, nullptr, const_cast<void*>(k_cache),
                                          const_cast<void*>(k_cache), const_cast<float*>(pyr),
-                                         const_cast<int32_t*>(len), sel, nullptr, nullptr, nullptr,
+                                         const_cast<int32_t*>(len), sel, nullptr, nullptr, nullptr, nullptr,
                                          as_stream(stream)));
   return from_cuda(launch_decode_rows(a, lay, 1, q_new, k_cache, nullptr, pyr, len, sel, nullptr, nullptr,
                                       as_stream(stream)));
@@ -213,24 +219,27 @@ pisa_status pisa_decode_select(const pisa_decode_config* cfg, const void* q_new,
 
 pisa_status pisa_decode_attn(const pisa_decode_config* cfg, const void* q_new, const void* k_cache,
                              const void* v_cache, const int32_t* len, const int32_t* sel, void* out, float* lse,
-                             void* stream) {
+                             void* workspace, void* stream) {
   pisa_status s = check_dcfg(cfg);
   if (s != PISA_OK) return s;
   if (!q_new || !k_cache || !v_cache || !len || !sel || !out) return PISA_ERR_INVALID_ARGUMENT;
   if (!aligned16(q_new) || !aligned16(k_cache) || !aligned16(v_cache)) return PISA_ERR_INVALID_ARGUMENT;
   const Layout lay = make_layout(cfg->cap, cfg->C);
   const DecodeArgs a = dargs_of(cfg);
-  if (decode_fused_supported(a))
+  if (decode_fused_supported(a)) {
+    if (!workspace || !aligned16(workspace)) return PISA_ERR_WORKSPACE;
     return from_cuda(launch_decode_fused(a, lay, 4, q_new, nullptr, nullptr, const_cast<void*>(k_cache),
                                          const_cast<void*>(v_cache), nullptr, const_cast<int32_t*>(len),
-                                         const_cast<int32_t*>(sel), out, lse, nullptr, as_stream(stream)));
+                                         const_cast<int32_t*>(sel), out, lse, nullptr,
+                                         static_cast<float*>(workspace), as_stream(stream)));
+  }
   return from_cuda(launch_decode_rows(a, lay, 2, q_new, k_cache, v_cache, nullptr, len, const_cast<int32_t*>(sel),
                                       out, lse, as_stream(stream)));
 }
 
 pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, const void* k_new, const void* v_new,
                              void* k_cache, void* v_cache, float* pyr, int32_t* len, int32_t* sel, void* out,
-                             float* lse, int32_t* status, void* stream) {
+                             float* lse, int32_t* status, void* workspace, void* stream) {
   pisa_status s = check_dcfg(cfg);
   if (s != PISA_OK) return s;
   if (!q_new || !k_new || !v_new || !k_cache || !v_cache || !pyr || !len || !out || !status)
@@ -239,9 +248,11 @@ pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, c
     return PISA_ERR_INVALID_ARGUMENT;
   const Layout lay = make_layout(cfg->cap, cfg->C);
   const DecodeArgs a = dargs_of(cfg);
-  if (decode_fused_supported(a))
+  if (decode_fused_supported(a)) {
+    if (!workspace || !aligned16(workspace)) return PISA_ERR_WORKSPACE;
     return from_cuda(launch_decode_fused(a, lay, 7, q_new, k_new, v_new, k_cache, v_cache, pyr, len, sel, out, lse,
-                                         status, as_stream(stream)));
+                                         status, static_cast<float*>(workspace), as_stream(stream)));
+  }
   cudaError_t e = launch_decode_append(a, lay, k_new, v_new, k_cache, v_cache, pyr, len, status, as_stream(stream));
   if (e != cudaSuccess) return PISA_ERR_CUDA;
   return from_cuda(

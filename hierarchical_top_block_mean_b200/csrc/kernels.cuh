@@ -44,9 +44,12 @@ cudaError_t launch_decode_rows(const DecodeArgs& a, const Layout& lay, int mode,
                                int32_t* sel, void* out, float* lse, cudaStream_t st);
 
 // Fused decode (bf16, H_kv <= 8, G_Q <= 8). mode bits: 1 append, 2 select, 4 attend.
+// lgt_ws: decode_logit_floats(a) floats, required when attending.
 bool decode_fused_supported(const DecodeArgs& a);
+int64_t decode_logit_floats(const DecodeArgs& a);
 cudaError_t launch_decode_fused(const DecodeArgs& a, const Layout& lay, int mode, const void* q_new,
                                 const void* k_new, const void* v_new, void* k_cache, void* v_cache, float* pyr,
-                                int32_t* len, int32_t* sel, void* out, float* lse, int32_t* status, cudaStream_t st);
+                                int32_t* len, int32_t* sel, void* out, float* lse, int32_t* status, float* lgt_ws,
+                                cudaStream_t st);
 
 }  // namespace pisa

@@ -198,6 +198,14 @@ pisa_status pisa_select_noalloc(const pisa_config* cfg, const void* q, const voi
  */
 int64_t pisa_decode_pyramid_rows(const pisa_decode_config* cfg);
 
+/* Bytes of device workspace that pisa_decode_attn and pisa_decode_step need
+ * (0 when the configuration needs none; 0 also for an invalid cfg). The
+ * fused kernel keeps there, per (sequence, kv head), the scaled logits
+ * scale q.k of the keys of up to 2K leaf blocks (fp32, [2K][C][G_Q]), so the
+ * attention reuses the leaf scorer's products instead of reading K again.
+ * Owned by the caller; contents need no initialisation and are scratch. */
+int64_t pisa_decode_workspace_bytes(const pisa_decode_config* cfg);
+
 /* Builds every sequence's pyramid over its first len[s] cached keys. */
 pisa_status pisa_decode_init(const pisa_decode_config* cfg, const void* k_cache, float* pyr, const int32_t* len,
                              void* stream);
@@ -213,16 +221,19 @@ pisa_status pisa_decode_select(const pisa_decode_config* cfg, const void* q_new,
                                const float* pyr, const int32_t* len, int32_t* sel, void* stream);
 
 /* Attention of q_new over the selected blocks of each sequence's first
- * len[s] tokens. out: [S, H_q, d] in dtype; lse: NULL or [S, H_q] fp32. */
+ * len[s] tokens. out: [S, H_q, d] in dtype; lse: NULL or [S, H_q] fp32.
+ * workspace: pisa_decode_workspace_bytes(cfg) bytes of device memory,
+ * 16-byte aligned (PISA_ERR_WORKSPACE when missing and needed). */
 pisa_status pisa_decode_attn(const pisa_decode_config* cfg, const void* q_new, const void* k_cache,
                              const void* v_cache, const int32_t* len, const int32_t* sel, void* out, float* lse,
-                             void* stream);
+                             void* workspace, void* stream);
 
 /* One decode step in one launch: append, select and attend for every
- * sequence. sel may be NULL (selection kept on chip); otherwise [S, H_kv, K]. */
+ * sequence. sel may be NULL (selection kept on chip); otherwise [S, H_kv, K].
+ * workspace: as for pisa_decode_attn. */
 pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, const void* k_new, const void* v_new,
                              void* k_cache, void* v_cache, float* pyr, int32_t* len, int32_t* sel, void* out,
-                             float* lse, int32_t* status, void* stream);
+                             float* lse, int32_t* status, void* workspace, void* stream);
 
 #ifdef __cplusplus
 }

@@ -102,4 +102,20 @@ def test_decode_validation():
     assert lib.pisa_decode_pyramid_rows(ctypes.byref(bad)) == 0
     ok = ctypes.c_void_p(256)
     assert lib.pisa_decode_append(ctypes.byref(dc), ok, ok, ok, ok, ok, ok, None, None) == 1  # status word required
-    assert lib.pisa_decode_step(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, ok, None, ok, None, ok, None) == 1
+    assert lib.pisa_decode_step(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, ok, None, ok, None, ok, ok, None) == 1
+    assert lib.pisa_decode_workspace_bytes(ctypes.byref(bad)) == 0
+
+
+def test_decode_workspace_size():
+    """The fused path keeps fp32 logits of 2K leaf blocks of C keys for the G_Q
+    heads of every (sequence, kv head); the fp32 fallback needs none."""
+    lib = _lib.lib()
+    S, cap, H_q, H_kv, d, C, K = 3, 4096, 16, 4, 128, 64, 16
+    bf = _lib.DecodeConfig(S, cap, H_q, H_kv, d, C, 2, K, 1, 0.0)
+    assert lib.pisa_decode_workspace_bytes(ctypes.byref(bf)) == S * H_kv * 2 * K * C * (H_q // H_kv) * 4
+    f32 = _lib.DecodeConfig(S, cap, H_q, H_kv, d, C, 2, K, 0, 0.0)
+    assert lib.pisa_decode_workspace_bytes(ctypes.byref(f32)) == 0
+    ok = ctypes.c_void_p(256)
+    # A needed workspace that is missing is refused before anything is enqueued.
+    assert lib.pisa_decode_step(ctypes.byref(bf), ok, ok, ok, ok, ok, ok, ok, None, ok, None, ok, None, None) == 3
+    assert lib.pisa_decode_attn(ctypes.byref(bf), ok, ok, ok, ok, ok, ok, None, None, None) == 3
