@@ -51,8 +51,8 @@ constexpr int kModeAppend = 1, kModeSelect = 2, kModeAttend = 4;
 constexpr int cmax(int x, int y) { return x > y ? x : y; }
 
 // Dynamic shared memory: the warps' tile rings during select and attend,
-// reused for the append's sibling rows and for the final merge of the warps'
-// softmax states.
+// reused for the append's sibling rows and leaf key rows and for the final
+// merge of the warps' softmax states.
 template <int D, int CC, int G>
 struct DecSmem {
   static constexpr int kTile = 16 * D;  // bf16 elements per ring tile
@@ -60,7 +60,8 @@ struct DecSmem {
   static constexpr int kState = 4 + 4 * (D / 16);  // m[2], l[2], o[D/16][4] per lane
   static constexpr int kMerge = kDecWarps * 32 * kState * 4;
   static constexpr int kSib = kMaxLevels * D * 4;
-  static constexpr int kBytes = cmax(kRing, cmax(kMerge, kSib));
+  static constexpr int kLeafOff = kSib;  // append: the leaf's key rows follow the siblings
+  static constexpr int kBytes = cmax(kRing, cmax(kMerge, kLeafOff + CC * D * 2));
 };
 
 struct TileSrc {
@@ -205,11 +206,24 @@ __global__ void __launch_bounds__(kDecWarps * 32, 4)
     const int64_t n = n0;  // position of the new token
     const int64_t leaf = n / C;
     const int L = num_levels(nn, C);
+    // The leaf's existing key rows are staged in shared memory by cp.async
+    // while the path's left siblings are read, so both cost one memory round
+    // trip; the new token's row is taken from k_new.
+    bf16* lrows = reinterpret_cast<bf16*>(dsm + SM::kLeafOff);  // [C][D]
+    const int64_t lo = leaf * C;
+    const int nold = static_cast<int>(n - lo);
+    for (int i = threadIdx.x; i < nold * (D / 8); i += blockDim.x) {
+      const int r = i / (D / 8), c8 = i % (D / 8);
+      cp_async16(lrows + r * D + c8 * 8, kh + (lo + r) * D + c8 * 8, 16);
+    }
+    cp_async_commit();
     if (warp == 0) {
       bf16* kr = kc + (bh * a.cap + n) * D;
       bf16* vr = vc + (bh * a.cap + n) * D;
       for (int e = lane; e < D / 2; e += 32) {
-        reinterpret_cast<uint32_t*>(kr)[e] = reinterpret_cast<const uint32_t*>(k_new + bh * D)[e];
+        const uint32_t kw = reinterpret_cast<const uint32_t*>(k_new + bh * D)[e];
+        reinterpret_cast<uint32_t*>(kr)[e] = kw;
+        reinterpret_cast<uint32_t*>(lrows + nold * D)[e] = kw;
         reinterpret_cast<uint32_t*>(vr)[e] = reinterpret_cast<const uint32_t*>(v_new + bh * D)[e];
       }
     }
@@ -220,11 +234,12 @@ __global__ void __launch_bounds__(kDecWarps * 32, 4)
       const int64_t c = leaf >> (l - 2);
       if (c & 1) buf[(l - 2) * D + e] = P[(off[l - 1] + c - 1) * D + e];
     }
+    cp_async_wait<0>();
     __threadfence_block();
     __syncthreads();
     if (warp == 0) {
       float mean[LM::kVec];
-      leaf_mean_warp<bf16, D>(kh, leaf * C, nn, mean);
+      leaf_mean_warp<bf16, D>(lrows, 0, nold + 1, mean);
       LM::store(mean, nullptr, P + (off[1] + leaf) * D, lane);
       for (int l = 2; l <= L; ++l) {
         const int64_t c = leaf >> (l - 2);
@@ -566,7 +581,7 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, const Layout& lay, int mode
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(a.S * a.H_kv));
     cfg.blockDim = dim3(kDecWarps * 32);
-    const int smem = DecSmem<D, 64, G>::kBytes;  // the same for both block sizes
+    const int smem = DecSmem<D, 64, G>::kBytes;  // covers both block sizes
     cudaError_t e0 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e0 != cudaSuccess) return e0;
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
