@@ -66,6 +66,8 @@ def _load():
             lib.oracle_select_rows.argtypes = [ctypes.POINTER(Cfg), p, p, p, i64, p, p, p, p, p, p, p]
             lib.oracle_select_flat_rows.restype = None
             lib.oracle_select_flat_rows.argtypes = [ctypes.POINTER(Cfg), p, p, i64, p, p, p]
+            lib.oracle_select_exact_rows.restype = None
+            lib.oracle_select_exact_rows.argtypes = [ctypes.POINTER(Cfg), p, p, i64, p, p, p]
             lib.oracle_attn_rows.restype = None
             lib.oracle_attn_rows.argtypes = [ctypes.POINTER(Cfg), p, p, p, i64, p, p, p, p]
             lib.oracle_decode_append.restype = None
@@ -169,6 +171,20 @@ def select_flat_rows(cfg: Cfg, q, pyr: np.ndarray, rows):
     sel = np.zeros((n, cfg.K), np.int32)
     gap = np.zeros(n, np.float64)
     _load().oracle_select_flat_rows(ctypes.byref(cfg), _ptr(qa), _ptr(pyr), n, _ptr(r), _ptr(sel), _ptr(gap))
+    return sel, gap
+
+
+def select_exact_rows(cfg: Cfg, q, k, rows):
+    """Exact-score flat selector (every usable leaf scored by its raw-key LSE,
+    summed over the GQA group) for rows (b, kv head, t). Returns sel [n, K]
+    and the K-th minus (K+1)-th score gap per row (inf when kept unscored)."""
+    qa, _ = _storage(q)
+    ka, _ = _storage(k)
+    r = _rows(rows)
+    n = r.shape[0]
+    sel = np.zeros((n, cfg.K), np.int32)
+    gap = np.zeros(n, np.float64)
+    _load().oracle_select_exact_rows(ctypes.byref(cfg), _ptr(qa), _ptr(ka), n, _ptr(r), _ptr(sel), _ptr(gap))
     return sel, gap
 
 

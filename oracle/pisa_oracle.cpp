@@ -344,6 +344,41 @@ void oracle_select_flat_rows(const oracle_cfg* c, const void* q, const double* p
   }
 }
 
+// Exact-score flat selector: the single-level block selection that the page
+// contrasts PISA with (§BSA: a flat method scores every block of the sequence;
+// §TopK: a block's score is the LSE of its raw keys). Every usable leaf gets
+// the pyramid selector's own leaf-level score,
+//   u_i = sum_{h' in group(h)} log sum_{j in leaf i, j usable} exp(scale q_{h',t} . k_j),
+// with the same validity, keep-all, tie and output rules. This is what the
+// coarse-to-fine search approximates: when the search scores every usable leaf
+// (M_1 <= 2K) the two coincide.
+void oracle_select_exact_rows(const oracle_cfg* c, const void* q, const void* k, int64_t n, const int64_t* rows,
+                              int32_t* sel, double* min_gap) {
+  const std::vector<int64_t> M = level_sizes(c->N, c->C);
+  const std::vector<int64_t> off = level_offsets(M);
+  const int64_t L = static_cast<int64_t>(M.size()) - 1;
+  const int64_t R = off[L + 1];
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t r = 0; r < n; ++r) {
+    const int64_t b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+    min_gap[r] = std::numeric_limits<double>::infinity();
+    std::vector<int64_t> V;
+    for (int64_t i = 0; i < M[1]; ++i)
+      if (valid_block(*c, M, 1, i, t)) V.push_back(i);
+    std::vector<int64_t> kept;
+    if (static_cast<int64_t>(V.size()) <= c->K) {
+      kept = V;
+    } else {
+      std::vector<std::pair<double, int64_t>> su;
+      for (int64_t i : V) su.emplace_back(block_score(*c, q, k, nullptr, M, off, R, b, h, t, 1, i), i);
+      kept = top_k(su, c->K, &min_gap[r]);
+    }
+    std::sort(kept.begin(), kept.end());
+    for (int64_t m = 0; m < c->K; ++m)
+      sel[r * c->K + m] = m < static_cast<int64_t>(kept.size()) ? static_cast<int32_t>(kept[m]) : -1;
+  }
+}
+
 // Block-sparse attention (§BSA):
 //   o_t = sum_{j in T_t} exp(q_t . k_j * scale) v_j / sum_{j in T_t} exp(q_t . k_j * scale)
 // over the raw keys and values of the selected leaf blocks, for every query

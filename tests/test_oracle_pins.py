@@ -383,6 +383,74 @@ def test_flat_selector_is_topk_of_dense_summary_scores(oracle, causal):
         assert list(sel[r][: len(want)]) == want
 
 
+# ------------------------------------------------------------ exact flat
+
+def _dense_block_lse_scores(x, w, b, h, t):
+    """All leaves' exact scores for one row from the dense score matrix: the
+    [G, N] logits of the group's heads (fp64), masked causally, split into
+    C-wide blocks (the ragged last one padded with -inf), logsumexp per block
+    (torch.logsumexp), summed over the heads."""
+    G = w.H_q // w.H_kv
+    q = x["q"][b, h * G:(h + 1) * G, t, :].double()
+    k = x["k"][b, h].double()
+    s = (q @ k.T) / math.sqrt(w.d)
+    if w.causal:
+        s[:, t + 1:] = -math.inf
+    M1 = -(-w.N // w.C)
+    pad = torch.full((G, M1 * w.C - w.N), -math.inf, dtype=s.dtype)
+    blocks = torch.cat([s, pad], dim=1).reshape(G, M1, w.C)
+    u = torch.logsumexp(blocks, dim=2).sum(0)
+    nv = (t // w.C + 1) if w.causal else M1
+    return u[:nv]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_selector_is_topk_of_dense_block_lse(oracle, causal):
+    # Exact single-level selection (§BSA scoring every block, with §TopK's LSE
+    # block score): the K largest dense block LSEs (torch.topk), ragged last
+    # leaf included (N = 1000 = 62 * 16 + 8).
+    w = _small(N=1000, C=16, K=5, causal=causal, H_q=6, H_kv=2, d=32, seed=5)
+    x = workloads.prefill_inputs(w)
+    cfg = _cfg(oracle, w)
+    rows = [(0, h, t) for h in range(2) for t in range(0, w.N, 7)]
+    sel, gap = oracle.select_exact_rows(cfg, x["q"], x["k"], rows)
+    for r, (b, h, t) in enumerate(rows):
+        u = _dense_block_lse_scores(x, w, b, h, t)
+        if u.numel() <= w.K:
+            want = list(range(u.numel()))
+            assert gap[r] == math.inf
+        else:
+            top = torch.topk(u, w.K + 1)
+            want = sorted(top.indices[: w.K].tolist())
+            assert gap[r] == pytest.approx((top.values[w.K - 1] - top.values[w.K]).item(), abs=1e-9)
+        assert list(sel[r][: len(want)]) == want
+        assert all(v == -1 for v in sel[r][len(want):])
+
+
+def test_exact_selector_equals_pyramid_when_every_leaf_is_scored(oracle):
+    # With M_2 <= K < M_1 the coarse-to-fine search starts at the leaf level
+    # and scores every usable leaf, so it must return the exact selection.
+    w = _small(N=512, C=16, K=16, causal=True, H_q=4, H_kv=2, d=16, seed=9)  # M_1 = 32, M_2 = 16
+    x = workloads.prefill_inputs(w)
+    cfg = _cfg(oracle, w)
+    pyr = oracle.build_pyramid(x["k"], w.C)
+    rows = [(0, h, t) for h in range(2) for t in range(0, w.N, 3)]
+    s_pyr, _ = oracle.select_rows(cfg, x["q"], x["k"], pyr, rows)
+    s_ex, _ = oracle.select_exact_rows(cfg, x["q"], x["k"], rows)
+    assert np.array_equal(s_pyr, s_ex)
+
+
+def test_exact_selector_finds_planted_needles(oracle):
+    w = workloads.Prefill("needle_small", B=1, N=4096, H_q=8, H_kv=2, d=64, C=32, K=4, causal=True,
+                          dtype="bf16", structure="needle", n_needles=24, seed=11)
+    x = workloads.prefill_inputs(w)
+    cfg = _cfg(oracle, w)
+    rows = [(0, h, t) for (t, j) in x["needles"] for h in range(w.H_kv)]
+    sel, _ = oracle.select_exact_rows(cfg, x["q"], x["k"], rows)
+    want = [j for (t, j) in x["needles"] for h in range(w.H_kv)]
+    assert all(j in list(s) for s, j in zip(sel, want))
+
+
 # ------------------------------------------------------------------ decode
 
 def test_decode_incremental_pyramid_equals_batch(oracle):
