@@ -155,6 +155,32 @@ def pyramid_bytes(w) -> float:
     return w.B * w.H_kv * (w.N * w.d * e + R * w.d * 4)
 
 
+def recall_at_k(sel, ref, chunk=1 << 16):
+    """Mean over rows of |sel_row & ref_row| / |ref_row| for [..., K] index
+    tensors padded with -1 (computed on the device in row chunks)."""
+    a = sel.reshape(-1, sel.shape[-1])
+    b = ref.reshape(-1, ref.shape[-1])
+    hit = 0
+    tot = 0
+    for i in range(0, a.shape[0], chunk):
+        x, y = a[i:i + chunk], b[i:i + chunk]
+        eq = (x[:, :, None] == y[:, None, :]) & (y[:, None, :] >= 0)
+        hit += int(eq.any(1).sum().item())
+        tot += int((y >= 0).sum().item())
+    return hit / max(tot, 1)
+
+
+def needle_recall(sel, needles):
+    """Share of planted (query position t, leaf j) needles, over every batch
+    row and kv head, whose leaf j is among the K selected for t."""
+    if not needles:
+        return None
+    ts = torch.tensor([t for t, _ in needles], device=sel.device)
+    js = torch.tensor([j for _, j in needles], device=sel.device, dtype=sel.dtype)
+    got = sel[:, :, ts, :]  # [B, H_kv, n, K]
+    return float((got == js[None, None, :, None]).any(-1).float().mean().item())
+
+
 def measured_traffic(workload: str, kernel: str):
     """DRAM bytes per launch of `kernel` recorded by an ncu capture in
     profiles/traffic.json, or None when absent or when any of the kernel's
@@ -315,6 +341,21 @@ def run_gpu(args):
     ms, value = aggregate(dist, dev_ms, w.B * w.N)
     stage_ms = {kk: vv / args.steps for kk, vv in stage.items()}
 
+    # Exact-score flat selector (every usable leaf scored by its raw-key LSE)
+    # on the same inputs, once after a warm-up, and the share of its top-K
+    # leaves that the pyramid search keeps.
+    pisa_sel = p.sel.clone()
+    xsel = api.select_exact(q, k, C=w.C, K=w.K, causal=w.causal)
+    xe0, xe1 = events(2)
+    xe0.record(stream)
+    api.select_exact(q, k, C=w.C, K=w.K, causal=w.causal, out=xsel)
+    xe1.record(stream)
+    torch.cuda.synchronize()
+    exact_ms = xe0.elapsed_time(xe1)
+    recall = recall_at_k(pisa_sel, xsel)
+    needles = {"pisa": needle_recall(pisa_sel, x["needles"]), "exact": needle_recall(xsel, x["needles"])}
+    del pisa_sel, xsel
+
     # Flat single-level selector on the same inputs (its own launches).
     fe0, fe1 = events(2)
     api.select_flat(q, p.pyr, C=w.C, K=w.K, causal=w.causal, H_kv=w.H_kv)
@@ -324,6 +365,7 @@ def run_gpu(args):
     fe1.record(stream)
     torch.cuda.synchronize()
     flat_ms = fe0.elapsed_time(fe1) / args.steps
+    needles["flat"] = needle_recall(p.sel, x["needles"])
 
     # End to end through the public API from pinned host buffers.
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
@@ -373,6 +415,10 @@ def run_gpu(args):
                    "l2": "inputs larger than L2 (q alone is %.0f MB)" % (q.numel() * q.element_size() / 1e6)},
         "stages_ms": stage_ms, "flat_select_ms": flat_ms,
         "select_speedup_vs_flat": flat_ms / stage_ms["select"] if stage_ms["select"] > 0 else None,
+        "exact_select_ms": exact_ms,
+        "select_speedup_vs_exact": exact_ms / stage_ms["select"] if stage_ms["select"] > 0 else None,
+        "pisa_recall_vs_exact": recall,
+        "needle_recall": needles if x["needles"] else None,
         "decode": decode,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

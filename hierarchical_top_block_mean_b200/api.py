@@ -138,6 +138,18 @@ def select_flat(q, pyr, *, C: int, K: int, causal: bool, H_kv: int, scale: float
     return out
 
 
+def select_exact(q, k, *, C: int, K: int, causal: bool, scale: float = 0.0, out=None):
+    """Exact-score flat top-K: every usable leaf scored by its raw-key LSE
+    summed over the group. sel [B, H_kv, N, K] int32."""
+    _need(q, "q")
+    _need(k, "k", q.dtype)
+    pr = Problem.of(q, k, C=C, K=K, causal=causal, scale=scale)
+    if out is None:
+        out = torch.empty((pr.B, pr.H_kv, pr.N, K), dtype=torch.int32, device=q.device)
+    _lib.call("pisa_select_exact", ctypes.byref(pr.cstruct()), _p(q), _p(k), _p(out), _stream(q))
+    return out
+
+
 def sparse_attn_fwd(q, k, v, sel, *, C: int, causal: bool, scale: float = 0.0, out=None, lse=None,
                     want_lse: bool = True):
     """Block-sparse attention over the selected leaf blocks: (out [B,H_q,N,d], lse [B,H_q,N] or None)."""

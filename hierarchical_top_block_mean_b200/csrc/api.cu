@@ -154,6 +154,15 @@ pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float*
   return from_cuda(launch_flat_rows(args_of(cfg), q, pyr, lay.R, sel, as_stream(stream)));
 }
 
+pisa_status pisa_select_exact(const pisa_config* cfg, const void* q, const void* k, int32_t* sel, void* stream) {
+  pisa_status s = check_cfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!q || !k || !sel || !aligned16(q) || !aligned16(k) || !aligned16(sel)) return PISA_ERR_INVALID_ARGUMENT;
+  const PrefillArgs a = args_of(cfg);
+  if (exact_umma_supported(a)) return from_cuda(launch_exact_umma(a, q, k, sel, as_stream(stream)));
+  return from_cuda(launch_exact_rows(a, q, k, sel, as_stream(stream)));
+}
+
 pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
                                  const int32_t* sel, void* out, float* lse, void* stream) {
   pisa_status s = check_cfg(cfg);

@@ -43,6 +43,11 @@ cudaError_t launch_decode_rows(const DecodeArgs& a, const Layout& lay, int mode,
                                const void* k_cache, const void* v_cache, const float* pyr, const int32_t* len,
                                int32_t* sel, void* out, float* lse, cudaStream_t st);
 
+// ---- exact-score flat selection (every usable leaf scored by its raw-key LSE)
+cudaError_t launch_exact_rows(const PrefillArgs& a, const void* q, const void* k, int32_t* sel, cudaStream_t st);
+bool exact_umma_supported(const PrefillArgs& a);
+cudaError_t launch_exact_umma(const PrefillArgs& a, const void* q, const void* k, int32_t* sel, cudaStream_t st);
+
 // Fused decode (bf16, H_kv <= 8, G_Q <= 8). mode bits: 1 append, 2 select, 4 attend.
 // lgt_ws: decode_logit_floats(a) floats, required when attending.
 bool decode_fused_supported(const DecodeArgs& a);

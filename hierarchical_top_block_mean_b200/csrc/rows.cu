@@ -123,6 +123,42 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   if (lane < a.K) sel[row * a.K + lane] = idx == INT_MAX ? -1 : idx;
 }
 
+// Exact-score flat selection for one row: every usable leaf is scored by its
+// raw-key LSE summed over the group (the pyramid search's leaf score), 32
+// leaves per round (one per lane), merged into the running best list.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kRowWarps * 32)
+    exact_rows_kernel(const T* __restrict__ q, const T* __restrict__ k, PrefillArgs a, int32_t* __restrict__ sel) {
+  __shared__ __align__(16) float qs[kRowWarps][G][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowWarps + warp;
+  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.N) return;
+  const int64_t bh = row / a.N, t = row % a.N;
+  const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
+  stage_q<T, D, G>(q + ((b * a.H_q + h * G) * a.N + t) * D, static_cast<int64_t>(a.N) * D, &qs[warp][0][0]);
+  SelectRow<T, D, G> sr{&qs[warp][0][0], nullptr, nullptr, k + bh * a.N * D, a.N, t, a.C, a.K,
+                        a.causal != 0, a.scale, nullptr};
+  const int64_t nv = valid_count(a.N, a.C, 1, t, a.causal != 0);
+  int idx;
+  if (nv <= a.K) {
+    idx = lane < nv ? lane : INT_MAX;
+  } else {
+    float bs = -INFINITY;
+    int bi = INT_MAX;
+    for (int64_t i0 = 0; i0 < nv; i0 += 32) {
+      float s = -INFINITY;
+      for (int x = 0; x < 32 && i0 + x < nv; ++x) {
+        const float u = sr.leaf_score(i0 + x);
+        if (lane == x) s = u;
+      }
+      warp_merge_best(bs, bi, s, i0 + lane < nv ? static_cast<int>(i0 + lane) : INT_MAX);
+    }
+    idx = lane < a.K ? bi : INT_MAX;
+  }
+  warp_sort_asc(idx);
+  if (lane < a.K) sel[row * a.K + lane] = idx == INT_MAX ? -1 : idx;
+}
+
 inline unsigned row_blocks(const PrefillArgs& a) {
   return static_cast<unsigned>((static_cast<int64_t>(a.B) * a.H_kv * a.N + kRowWarps - 1) / kRowWarps);
 }
@@ -160,6 +196,17 @@ cudaError_t launch_flat_rows(const PrefillArgs& a, const void* q, const float* p
     using T = typename decltype(tt)::type;
     constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
     flat_rows_kernel<T, D, G><<<row_blocks(a), kRowWarps * 32, 0, st>>>(static_cast<const T*>(q), pyr, R, a, sel);
+    count_launch();
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_exact_rows(const PrefillArgs& a, const void* q, const void* k, int32_t* sel, cudaStream_t st) {
+  return dispatch_tdg(a.dtype, a.d, a.H_q / a.H_kv, [&](auto tt, auto dd, auto gg) -> cudaError_t {
+    using T = typename decltype(tt)::type;
+    constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
+    exact_rows_kernel<T, D, G><<<row_blocks(a), kRowWarps * 32, 0, st>>>(static_cast<const T*>(q),
+                                                                          static_cast<const T*>(k), a, sel);
     count_launch();
     return cudaGetLastError();
   });

@@ -142,6 +142,20 @@ pisa_status pisa_select(const pisa_config* cfg, const void* q, const void* k, co
 pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float* pyr, int32_t* sel, void* stream);
 
 /*
+ * Exact-score flat selection — the single-level block selection that the
+ * pyramid search approximates (§BSA: a flat method scores every block; §TopK:
+ * a block's score is the LSE of its raw keys). Every usable leaf is scored by
+ *   u_i = sum over the group of log sum_{j in leaf i, j usable} exp(scale q_{h',t} . k_j)
+ * (the pyramid search's leaf-level score) and the top K are kept with the same
+ * validity, keep-all, tie, order and padding rules as pisa_select. Work is
+ * O(N^2 d) per kv head; needs no pyramid and no workspace.
+ *   q : [B, H_q, N, d];  k : [B, H_kv, N, d];  sel : [B, H_kv, N, K] int32.
+ * bf16 with d = 128 and C = 64 runs on tcgen05 tensor cores; other
+ * configurations on a warp-per-row kernel.
+ */
+pisa_status pisa_select_exact(const pisa_config* cfg, const void* q, const void* k, int32_t* sel, void* stream);
+
+/*
  * Block-sparse attention forward — §BSA:
  *   o_t = sum_{j in T_t} exp(scale q_t.k_j) v_j / sum_{j in T_t} exp(scale q_t.k_j)
  * over the raw keys of the selected leaf blocks T_t (shared by the query heads
