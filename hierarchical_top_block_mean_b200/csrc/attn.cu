@@ -4,8 +4,9 @@
 // group at once.
 //
 // Each warp owns one (kv head, query) row at a time and streams the row's
-// selected blocks through its own double-buffered shared-memory ring, in
-// chunks of kKeysPerChunk keys (K and V rows). One lane issues the chunk as
+// selected blocks through its own ring of kAttnStages shared-memory stages,
+// in chunks of kKeysPerChunk keys (K and V rows), kAttnStages - 1 chunks in
+// flight while one is in use. One lane issues the chunk as
 // bulk tensor copies (TMA: chunk-row x 64-column boxes with the hardware
 // 128-byte swizzle) that complete on the stage's mbarrier, so the copy costs
 // the warp a handful of instructions and ldmatrix reads are conflict-free.
@@ -26,12 +27,15 @@ namespace pisa {
 namespace {
 
 constexpr int kAttnWarps = 12;
+constexpr int kAttnStages = 2;
 constexpr int kKeysPerChunk = 16;
+constexpr float kLazy = 8.f;  // headroom of the lazily moved softmax maximum (natural-log units)
 
 // Work cursor of one warp: row, the row's selected blocks (compacted, one
 // per lane, held in a register), position in that list and chunk.
 struct Cursor {
   int64_t row;  // -1: exhausted
+  int bh, t;    // row = bh * N + t (divided once per row)
   int blk_lane; // this lane's entry of the row's compacted block list
   int nblk;     // blocks in the list
   int idx;      // position in the list
@@ -48,15 +52,14 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   constexpr int kHalves = CC / kKeysPerChunk;  // chunks per leaf block
   constexpr int kMT = kKeysPerChunk / 16;      // 16-key M tiles per chunk
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ uint64_t bars[kAttnWarps][2];
+  __shared__ uint64_t bars[kAttnWarps][kAttnStages];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   // 128-byte swizzled boxes need 1 KB alignment.
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* ring = smem + warp * (2 * 2 * kChunkBytes);  // [stage][K|V][chunk]
+  unsigned char* ring = smem + warp * (kAttnStages * 2 * kChunkBytes);  // [stage][K|V][chunk]
   if (lane == 0) {
-    mbar_init(&bars[warp][0], 1);
-    mbar_init(&bars[warp][1], 1);
+    for (int i = 0; i < kAttnStages; ++i) mbar_init(&bars[warp][i], 1);
     mbar_init_fence();
   }
   __syncwarp();
@@ -83,13 +86,14 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
           }
         }
       }
-      return Cursor{r, out_b, __popc(m), 0, 0};
+      return Cursor{r, static_cast<int>(r / n), static_cast<int>(r % n), out_b, __popc(m), 0, 0};
     }
-    return Cursor{-1, -1, 0, 0, 0};
+    return Cursor{-1, 0, 0, -1, 0, 0, 0};
   };
   auto advance = [&](const Cursor& c) -> Cursor {
-    if (c.half + 1 < kHalves) return Cursor{c.row, c.blk_lane, c.nblk, c.idx, c.half + 1};
-    if (c.idx + 1 < c.nblk) return Cursor{c.row, c.blk_lane, c.nblk, c.idx + 1, 0};
+    if (c.row < 0) return c;
+    if (c.half + 1 < kHalves) return Cursor{c.row, c.bh, c.t, c.blk_lane, c.nblk, c.idx, c.half + 1};
+    if (c.idx + 1 < c.nblk) return Cursor{c.row, c.bh, c.t, c.blk_lane, c.nblk, c.idx + 1, 0};
     return load_row(c.row + stride);
   };
   // Issues chunk c into ring stage st: K and V rows [key0, key0 + 32) of
@@ -99,8 +103,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     if (c.row < 0) return;
     const int blk = __shfl_sync(kFull, c.blk_lane, c.idx);
     if (lane == 0) {
-      const int64_t bh = c.row / n;
-      const int y = static_cast<int>(bh * n + static_cast<int64_t>(blk) * CC + c.half * kKeysPerChunk);
+      const int y = static_cast<int>(c.bh * n + static_cast<int64_t>(blk) * CC + c.half * kKeysPerChunk);
       unsigned char* ks = ring + st * 2 * kChunkBytes;
       unsigned char* vs = ks + kChunkBytes;
       fence_proxy_async();  // the stage's previous contents were read by ldmatrix
@@ -113,24 +116,35 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     }
   };
 
+  // Chunks are issued in order, chunk c into stage c mod kAttnStages; tail is
+  // the last one issued.
   Cursor cur = load_row(static_cast<int64_t>(blockIdx.x) * kAttnWarps + warp);
   issue(cur, 0);
+  Cursor tail = cur;
+#pragma unroll
+  for (int i = 1; i < kAttnStages - 1; ++i) {
+    tail = advance(tail);
+    issue(tail, i);
+  }
   int st = 0;
   int64_t row_now = -1;
   uint32_t qb[kKS][2];
   float m[2], l[2], o[kKS][4];
+  int hb = 0, hh = 0;  // batch and kv head of the current row
 
   while (cur.row >= 0) {
     const Cursor nxt = advance(cur);
-    issue(nxt, st ^ 1);
+    tail = kAttnStages == 2 ? nxt : advance(tail);
+    issue(tail, st == 0 ? kAttnStages - 1 : st - 1);  // the stage read in the previous iteration
     mbar_wait(&bars[warp][st], (phase >> st) & 1u, faults);
     phase ^= 1u << st;
 
-    const int64_t bh = cur.row / n, t = cur.row % n;
-    const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
+    const int64_t t = cur.t;
     if (cur.row != row_now) {  // first chunk of a row: queries and softmax state
+      hb = cur.bh / a.H_kv;
+      hh = cur.bh % a.H_kv;
       row_now = cur.row;
-      const bf16* qp = q + ((b * a.H_q + h * G + (gid < G ? gid : 0)) * n + t) * D + 2 * tig;
+      const bf16* qp = q + ((static_cast<int64_t>(hb) * a.H_q + hh * G + (gid < G ? gid : 0)) * n + t) * D + 2 * tig;
 #pragma unroll
       for (int ks = 0; ks < kKS; ++ks) {
         qb[ks][0] = gid < G ? *reinterpret_cast<const uint32_t*>(qp + 16 * ks) : 0u;
@@ -141,10 +155,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 #pragma unroll
       for (int i = 0; i < kKS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     }
-    int64_t last = n - 1;
-    if (causal && t < last) last = t;
+    const int last = (causal && cur.t < n - 1) ? cur.t : static_cast<int>(n - 1);  // positions fit int32
     const int blk = __shfl_sync(kFull, cur.blk_lane, cur.idx);
-    const int64_t key0 = static_cast<int64_t>(blk) * CC + cur.half * kKeysPerChunk;
+    const int key0 = blk * CC + cur.half * kKeysPerChunk;
     const bool full = key0 + kKeysPerChunk - 1 <= last;
     const unsigned char* ks_ = ring + st * 2 * kChunkBytes;
     const unsigned char* vs_ = ks_ + kChunkBytes;
@@ -182,17 +195,29 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
           bm[j] = fmaxf(bm[j], x);
         }
       }
-    float alpha[2], mn[2];
+    // Lazy rescaling: the reference maximum m of a head moves only when one
+    // of its logits exceeds m by more than kLazy; o and the partial sums are
+    // then rescaled. Otherwise p = exp(x - m) <= e^kLazy, which fp32 and the
+    // bf16 P operand hold at full relative precision, and the chunk needs no
+    // cross-lane reduction. Row sums are kept per lane and reduced at the end
+    // of the row.
+    if (__any_sync(kFull, bm[0] > m[0] + kLazy || bm[1] > m[1] + kLazy)) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      bm[j] = fmaxf(bm[j], __shfl_xor_sync(kFull, bm[j], 4));
-      bm[j] = fmaxf(bm[j], __shfl_xor_sync(kFull, bm[j], 8));
-      bm[j] = fmaxf(bm[j], __shfl_xor_sync(kFull, bm[j], 16));
-      mn[j] = fmaxf(m[j], bm[j]);
-      alpha[j] = (m[j] == -INFINITY) ? 0.f : expf(m[j] - mn[j]);
-      m[j] = mn[j];
+      for (int j = 0; j < 2; ++j) {
+        bm[j] = fmaxf(bm[j], __shfl_xor_sync(kFull, bm[j], 4));
+        bm[j] = fmaxf(bm[j], __shfl_xor_sync(kFull, bm[j], 8));
+        bm[j] = fmaxf(bm[j], __shfl_xor_sync(kFull, bm[j], 16));
+        const float mn = fmaxf(m[j], bm[j]);
+        const float alpha = (m[j] == -INFINITY) ? 0.f : expf(m[j] - mn);
+        m[j] = mn;
+        l[j] *= alpha;
+#pragma unroll
+        for (int md = 0; md < kKS; ++md) {
+          o[md][j] *= alpha;
+          o[md][2 + j] *= alpha;
+        }
+      }
     }
-    float ps[2] = {0.f, 0.f};
     uint32_t pb[kMT][2];
 #pragma unroll
     for (int mt = 0; mt < kMT; ++mt) {
@@ -200,25 +225,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int j = i & 1;
-        p[i] = (s[mt][i] == -INFINITY) ? 0.f : expf(s[mt][i] - mn[j]);
-        ps[j] += p[i];
+        p[i] = (s[mt][i] == -INFINITY) ? 0.f : expf(s[mt][i] - m[j]);
+        l[j] += p[i];
       }
       pb[mt][0] = movtrans(pack_bf16(p[0], p[1]));
       pb[mt][1] = movtrans(pack_bf16(p[2], p[3]));
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      ps[j] += __shfl_xor_sync(kFull, ps[j], 4);
-      ps[j] += __shfl_xor_sync(kFull, ps[j], 8);
-      ps[j] += __shfl_xor_sync(kFull, ps[j], 16);
-      l[j] = l[j] * alpha[j] + ps[j];
-    }
-#pragma unroll
-    for (int md = 0; md < kKS; ++md) {
-      o[md][0] *= alpha[0];
-      o[md][1] *= alpha[1];
-      o[md][2] *= alpha[0];
-      o[md][3] *= alpha[1];
     }
     // ---- O^T += V^T P^T (one k step per 16 keys)
 #pragma unroll
@@ -235,8 +246,14 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     __syncwarp();  // this stage is refilled by the next iteration's prefetch
 
     if (nxt.row != cur.row) {  // last chunk of the row: write o / l and lse
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        l[j] += __shfl_xor_sync(kFull, l[j], 4);
+        l[j] += __shfl_xor_sync(kFull, l[j], 8);
+        l[j] += __shfl_xor_sync(kFull, l[j], 16);
+      }
       const int64_t hs = n * D;
-      bf16* o0 = out + ((b * a.H_q + h * G) * n + t) * D;
+      bf16* o0 = out + ((static_cast<int64_t>(hb) * a.H_q + hh * G) * n + t) * D;
       float inv[2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) inv[j] = l[j] > 0.f ? 1.f / l[j] : 0.f;
@@ -252,11 +269,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       if (lse && gid == 0) {
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-          if (2 * tig + j < G) lse[(b * a.H_q + h * G + 2 * tig + j) * n + t] = m[j] + logf(l[j]);
+          if (2 * tig + j < G) lse[(static_cast<int64_t>(hb) * a.H_q + hh * G + 2 * tig + j) * n + t] = m[j] + logf(l[j]);
       }
     }
     cur = nxt;
-    st ^= 1;
+    st = st + 1 == kAttnStages ? 0 : st + 1;
   }
 }
 
@@ -285,7 +302,7 @@ cudaError_t launch_attn_mma(const PrefillArgs& a, const void* q, const void* k, 
   unsigned long long* faults = wait_fault_counter();
   return dispatch_tdg(PISA_DTYPE_BF16, a.d, a.H_q / a.H_kv, [&](auto, auto dd, auto gg) -> cudaError_t {
     constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
-    const size_t smem = static_cast<size_t>(kAttnWarps) * 2 * 2 * kKeysPerChunk * D * 2 + 1024;
+    const size_t smem = static_cast<size_t>(kAttnWarps) * kAttnStages * 2 * kKeysPerChunk * D * 2 + 1024;
     auto kern = a.C == 64 ? attn_kernel<D, 64, G> : attn_kernel<D, 32, G>;
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e2 != cudaSuccess) return e2;
