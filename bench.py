@@ -353,7 +353,8 @@ def run_gpu(args):
     torch.cuda.synchronize()
     exact_ms = xe0.elapsed_time(xe1)
     recall = recall_at_k(pisa_sel, xsel)
-    needles = {"pisa": needle_recall(pisa_sel, x["needles"]), "exact": needle_recall(xsel, x["needles"])}
+    needles = ({"pisa": needle_recall(pisa_sel, x["needles"]), "exact": needle_recall(xsel, x["needles"])}
+               if x["needles"] else None)
     del pisa_sel, xsel
 
     # Flat single-level selector on the same inputs (its own launches).
@@ -365,7 +366,8 @@ def run_gpu(args):
     fe1.record(stream)
     torch.cuda.synchronize()
     flat_ms = fe0.elapsed_time(fe1) / args.steps
-    needles["flat"] = needle_recall(p.sel, x["needles"])
+    if needles:
+        needles["flat"] = needle_recall(p.sel, x["needles"])
 
     # End to end through the public API from pinned host buffers.
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
@@ -418,7 +420,7 @@ def run_gpu(args):
         "exact_select_ms": exact_ms,
         "select_speedup_vs_exact": exact_ms / stage_ms["select"] if stage_ms["select"] > 0 else None,
         "pisa_recall_vs_exact": recall,
-        "needle_recall": needles if x["needles"] else None,
+        "needle_recall": needles,
         "decode": decode,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

@@ -26,7 +26,7 @@ namespace pisa {
 
 namespace {
 
-constexpr int kAttnWarps = 12;
+constexpr int kAttnWarps = 14;
 constexpr int kAttnStages = 2;
 constexpr int kKeysPerChunk = 16;
 constexpr float kLazy = 8.f;  // headroom of the lazily moved softmax maximum (natural-log units)

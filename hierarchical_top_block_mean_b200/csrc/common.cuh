@@ -26,7 +26,21 @@ void count_launch(int n = 1);
 // Pyramid level sizes (paper §Pyramid): M_1 = ceil(n / C), M_{l+1} =
 // ceil(M_l / 2). Because ceil(ceil(x / a) / b) = ceil(x / (a b)) for positive
 // integers, M_l = ceil(n / (C 2^(l-1))).
+// log2 of a power of two.
+__host__ __device__ inline int ilog2_pow2(int x) {
+#ifdef __CUDA_ARCH__
+  return __ffs(x) - 1;
+#else
+  return __builtin_ctz(static_cast<unsigned>(x));
+#endif
+}
+__host__ __device__ inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
 __host__ __device__ inline int64_t level_size(int64_t n, int C, int l) {
+  if (is_pow2(C)) {  // every block size the kernels support: a shift, not a 64-bit division
+    const int sh = ilog2_pow2(C) + l - 1;
+    return (n + (int64_t{1} << sh) - 1) >> sh;
+  }
   int64_t span = static_cast<int64_t>(C) << (l - 1);
   return (n + span - 1) / span;
 }
@@ -68,7 +82,7 @@ inline Layout make_layout(int64_t n_layout, int C) {
 __device__ inline int64_t valid_count(int64_t n, int C, int l, int64_t t, bool causal) {
   int64_t m = level_size(n, C, l);
   if (!causal) return m;
-  int64_t v = t / level_span(C, l) + 1;
+  int64_t v = (is_pow2(C) ? (t >> (ilog2_pow2(C) + l - 1)) : t / level_span(C, l)) + 1;
   return v < m ? v : m;
 }
 

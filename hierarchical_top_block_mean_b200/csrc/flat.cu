@@ -100,6 +100,10 @@ __global__ void __launch_bounds__(kFlatWarps * 32, 2)
       alo[ks][2 + half] = pack_bf16(ll[2], ll[3]);
     }
   }
+  // Usable leaves of this lane's two rows (causal: first key <= t).
+  int64_t lim[2];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) lim[half] = causal ? min(nleaf, trow[half] / a.C + 1) : nleaf;
   float thr[2] = {-INFINITY, -INFINITY};
   int thri[2] = {INT_MAX, INT_MAX};
   const int lr0 = 16 * warp + gid;
@@ -143,14 +147,13 @@ __global__ void __launch_bounds__(kFlatWarps * 32, 2)
     uint32_t cand = 0;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      const int64_t lim = causal ? min(nleaf, trow[half] / a.C + 1) : nleaf;
 #pragma unroll
       for (int nt = 0; nt < kChunk / 8; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int64_t i = c0 + 8 * nt + 2 * tig + e;
           acc[nt][2 * half + e] *= a.scale;
-          if (rok[half] && i < lim && ranks_before(acc[nt][2 * half + e], static_cast<int>(i), thr[half], thri[half]))
+          if (rok[half] && i < lim[half] && ranks_before(acc[nt][2 * half + e], static_cast<int>(i), thr[half], thri[half]))
             cand |= 1u << (16 * half + 2 * nt + e);
         }
     }

@@ -46,7 +46,7 @@ constexpr int kAccStages = 4;                           // TMEM accumulator buff
 constexpr uint32_t kTmemCols = kAccStages * kAccCols;
 
 struct Cursor2 {
-  int item, bucket, p_lo, p_hi, ntiles;
+  int item, bh, leaf, p_lo, p_hi, ntiles;
 };
 
 __global__ void __launch_bounds__(kUmmaThreads, 1)
@@ -85,14 +85,14 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   const uint32_t tmem = tmem_base_sh;
 
   const int total = ws.item_off[nb];
-  const int64_t bucket_span = static_cast<int64_t>(ws.nwin) * M1;
   const bool causal = a.causal != 0;
   // Work-item records are loaded one item ahead (one 16-byte load each).
   auto info = [&](int item) { return item < total ? ws.item_info[item] : make_int4(0, 0, 0, 0); };
   auto cursor = [&](int item, int4 inf) {
     Cursor2 c;
     c.item = item;
-    c.bucket = inf.x;
+    c.bh = inf.x;
+    c.leaf = inf.w;
     c.p_lo = inf.y;
     c.p_hi = inf.z;
     c.ntiles = (c.p_hi - c.p_lo + kTilePairs - 1) / kTilePairs;
@@ -111,8 +111,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
       const Cursor2 c = cursor(item, inf);
       inf = info(item + gridDim.x);
-      const int64_t bh = c.bucket / bucket_span;
-      const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
+      const int64_t b = c.bh / a.H_kv, h = c.bh % a.H_kv;
       const bf16* qg = q + (b * a.H_q + h * 8) * static_cast<int64_t>(a.N) * 128;  // head 0 of the group
       const bf16* qrow0 = qg + g0 * head_stride + jcol * 8;                        // this thread's column of head g0
       for (int tl = 0; tl < c.ntiles; ++tl) {
@@ -168,8 +167,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       auto load_key = [&](int4 ki, int n) {
         const int kbn = n & 1;
         mbar_wait(&kempty[kbn], ((n >> 1) & 1) ^ 1, faults);
-        const int64_t bhk = ki.x / bucket_span, leafk = ki.x % M1;
-        const int ky = static_cast<int>(bhk * a.N + leafk * 64);
+        const int ky = static_cast<int>(static_cast<int64_t>(ki.x) * a.N + static_cast<int64_t>(ki.w) * 64);
         fence_proxy_async();
         mbar_expect_tx(&kfull[kbn], kKeyBytes);
         tma_load_2d(kbuf + kbn * kKeyBytes, &tmk, 0, ky, &kfull[kbn]);
@@ -225,8 +223,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     while (item < total) {
       const uint32_t w = w_next;
       const bool ok = w != 0xffffffffu;
-      const int64_t bh = c.bucket / bucket_span;
-      const int64_t key0 = static_cast<int64_t>(c.bucket % M1) * 64;
+      const int64_t bh = c.bh;
+      const int64_t key0 = static_cast<int64_t>(c.leaf) * 64;
       const int nkeys = static_cast<int>(min(static_cast<int64_t>(64), a.N - key0));
       // Advance the stream and prefetch the next tile's word.
       Cursor2 cn = c;

@@ -302,15 +302,16 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ws ws, int64_t rows, int N
 }
 
 // Item -> (bucket, pair range) map: one thread per bucket writes its items' entries.
-__global__ void __launch_bounds__(256) itemize_kernel(Ws ws, int nb) {
+__global__ void __launch_bounds__(256) itemize_kernel(Ws ws, int nb, int M1) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= nb) return;
   const int i0 = ws.item_off[b], i1 = ws.item_off[b + 1];
   const int p0 = ws.bucket_off[b], p1 = ws.bucket_off[b + 1];
+  const int bh = b / (ws.nwin * M1), leaf = b % M1;  // bucket = (bh * nwin + window) * M1 + leaf
   for (int i = i0; i < i1; ++i) {
     ws.item_bucket[i] = b;
     const int lo = p0 + (i - i0) * kPairsPerItem;
-    ws.item_info[i] = make_int4(b, lo, min(lo + kPairsPerItem, p1), 0);
+    ws.item_info[i] = make_int4(bh, lo, min(lo + kPairsPerItem, p1), leaf);
   }
 }
 
@@ -591,7 +592,7 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   count_launch();
   scatter_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(ws, rows, a.N, M1);
   count_launch();
-  itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(ws, nb);
+  itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(ws, nb, M1);
   count_launch();
   if (leaf_umma_supported(a)) {
     if ((e = launch_leaf_umma(a, q, k, ws, nb, M1, st)) != cudaSuccess) return e;

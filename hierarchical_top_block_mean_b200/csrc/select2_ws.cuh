@@ -17,7 +17,7 @@ struct Ws {
   uint32_t* pairs;      // [rows * 32] (t << 5 | slot), grouped by bucket
   uint4* planes;        // [B*H_kv][R][D/4] pyramid rows as bf16 hi/lo: {hi x4, lo x4} per 4 elements
   int32_t* item_bucket; // [items] bucket of each stage-2 work item
-  int4* item_info;      // [items] {bucket, first pair, end pair, 0} of each work item
+  int4* item_info;      // [items] {b * H_kv + h, first pair, end pair, leaf} of each work item
   int win_shift;        // queries are bucketed by window t >> win_shift
   int nwin;             // windows per (b, kv head)
 };
