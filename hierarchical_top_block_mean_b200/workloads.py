@@ -98,6 +98,10 @@ PREFILL = {
                              dtype="bf16", structure="clustered", segment=4096, seed=3000),
     "needle_256k": Prefill("needle_256k", B=1, N=262144, H_q=16, H_kv=2, d=128, C=64, K=16, causal=True,
                            dtype="bf16", structure="needle", n_needles=256, seed=4000),
+    # The 256K head layout (G_Q = 8) at a quarter of the length: a profiling
+    # and parity case for the G_Q = 8 kernels that still exceeds L2 (q: 268 MB).
+    "needle_64k_g8": Prefill("needle_64k_g8", B=1, N=65536, H_q=16, H_kv=2, d=128, C=64, K=16, causal=True,
+                             dtype="bf16", structure="needle", n_needles=64, seed=4500),
 }
 
 DECODE = {

@@ -90,7 +90,8 @@ def test_large_K_prefill_equals_dense_attention():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,rows", [("needle_16k", 4096), ("clustered_64k", 2048), ("needle_256k", 1024)])
+@pytest.mark.parametrize("name,rows", [("needle_16k", 4096), ("clustered_64k", 2048), ("needle_64k_g8", 2048),
+                                       ("needle_256k", 1024)])
 def test_prefill_parity_full_size(name, rows):
     w = workloads.PREFILL[name]
     r = _run(w, rows)
