@@ -161,14 +161,20 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
             x0[ks] = __ldg(p0 + 4 * ks);
             x1[ks] = __ldg(p1 + 4 * ks);
           }
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          // Four accumulators (hi / lo x even / odd k step) keep the MMA
+          // dependency chains short.
+          float ah0[4] = {0.f, 0.f, 0.f, 0.f}, ah1[4] = {0.f, 0.f, 0.f, 0.f};
+          float al0[4] = {0.f, 0.f, 0.f, 0.f}, al1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
             const uint32_t hi[4] = {x0[ks].x, x1[ks].x, x0[ks].y, x1[ks].y};
             const uint32_t lo[4] = {x0[ks].z, x1[ks].z, x0[ks].w, x1[ks].w};
-            mma_bf16(acc, hi, qb[ks][0], qb[ks][1]);
-            mma_bf16(acc, lo, qb[ks][0], qb[ks][1]);
+            mma_bf16((ks & 1) ? ah1 : ah0, hi, qb[ks][0], qb[ks][1]);
+            mma_bf16((ks & 1) ? al1 : al0, lo, qb[ks][0], qb[ks][1]);
           }
+          float acc[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = (ah0[i] + ah1[i]) + (al0[i] + al1[i]);
           // acc: [first child, head 2tig], [first, 2tig+1], [second, 2tig], [second, 2tig+1]
           float u = 0.f;
 #pragma unroll
