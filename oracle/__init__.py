@@ -67,6 +67,8 @@ def _load():
             lib.oracle_select_flat_rows.restype = None
             lib.oracle_select_flat_rows.argtypes = [ctypes.POINTER(Cfg), p, p, i64, p, p, p]
             lib.oracle_select_exact_rows.restype = None
+            lib.oracle_attn_bwd.restype = None
+            lib.oracle_attn_bwd.argtypes = [ctypes.POINTER(Cfg), p, p, p, p, p, p, p, p]
             lib.oracle_select_exact_rows.argtypes = [ctypes.POINTER(Cfg), p, p, i64, p, p, p]
             lib.oracle_attn_rows.restype = None
             lib.oracle_attn_rows.argtypes = [ctypes.POINTER(Cfg), p, p, p, i64, p, p, p, p]
@@ -202,6 +204,23 @@ def attn_rows(cfg: Cfg, q, k, v, rows, sel):
     lse = np.zeros((n, G), np.float64)
     _load().oracle_attn_rows(ctypes.byref(cfg), _ptr(qa), _ptr(ka), _ptr(va), n, _ptr(r), _ptr(s), _ptr(out), _ptr(lse))
     return out, lse
+
+
+def attn_bwd(cfg: Cfg, q, k, v, sel, dout):
+    """Gradient of the block-sparse attention with the selection sel
+    [B, H_kv, N, K] held fixed: returns dq [B, H_q, N, d], dk, dv
+    [B, H_kv, N, d] (fp64) for the output gradient dout [B, H_q, N, d]."""
+    qa, _ = _storage(q)
+    ka, _ = _storage(k)
+    va, _ = _storage(v)
+    ga, _ = _storage(dout)
+    s = np.ascontiguousarray(np.asarray(sel, dtype=np.int32))
+    dq = np.zeros((cfg.B, cfg.H_q, cfg.N, cfg.d), np.float64)
+    dk = np.zeros((cfg.B, cfg.H_kv, cfg.N, cfg.d), np.float64)
+    dv = np.zeros((cfg.B, cfg.H_kv, cfg.N, cfg.d), np.float64)
+    _load().oracle_attn_bwd(ctypes.byref(cfg), _ptr(qa), _ptr(ka), _ptr(va), _ptr(s), _ptr(ga), _ptr(dq), _ptr(dk),
+                            _ptr(dv))
+    return dq, dk, dv
 
 
 def decode_append(seq_keys, n: int, C: int, cap: int, pyr: np.ndarray) -> None:

@@ -422,6 +422,83 @@ void oracle_attn_rows(const oracle_cfg* c, const void* q, const void* k, const v
   }
 }
 
+// Gradient of the block-sparse attention (§BSA) with the selection held
+// fixed: the selection is a discrete choice, so only the attention over the
+// selected keys is differentiated. For every row (b, kv head h, t) and query
+// head h' of the group, over the row's usable keys j (the union of its
+// selected blocks; causal: j <= t), with dout the gradient of o:
+//   s_j = scale q.k_j,  P_j = exp(s_j) / sum_i exp(s_i),  o = sum_j P_j v_j,
+//   dP_j = dout . v_j,  D = dout . o,  dS_j = P_j (dP_j - D),
+//   dq += scale sum_j dS_j k_j,  dk_j += scale dS_j q,  dv_j += P_j dout.
+// Every row of the problem is processed (the key gradients sum over rows).
+// q, dout: [B, H_q, N, d]; k, v: [B, H_kv, N, d]; sel: [B, H_kv, N, K].
+// dq: [B, H_q, N, d]; dk, dv: [B, H_kv, N, d]; fp64, overwritten.
+void oracle_attn_bwd(const oracle_cfg* c, const void* q, const void* k, const void* v, const int32_t* sel,
+                     const void* dout, double* dq, double* dk, double* dv) {
+  const int64_t G = c->H_q / c->H_kv;
+  const double sc = cfg_scale(*c);
+  const int64_t d = c->d;
+  std::fill(dq, dq + c->B * c->H_q * c->N * d, 0.0);
+  std::fill(dk, dk + c->B * c->H_kv * c->N * d, 0.0);
+  std::fill(dv, dv + c->B * c->H_kv * c->N * d, 0.0);
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t bh = 0; bh < c->B * c->H_kv; ++bh) {  // one kv head owns its dk, dv
+    const int64_t b = bh / c->H_kv, h = bh % c->H_kv;
+    for (int64_t t = 0; t < c->N; ++t) {
+      const int32_t* srow = sel + (bh * c->N + t) * c->K;
+      std::vector<int64_t> blocks;
+      for (int64_t m = 0; m < c->K; ++m)
+        if (srow[m] >= 0) blocks.push_back(srow[m]);
+      std::sort(blocks.begin(), blocks.end());
+      blocks.erase(std::unique(blocks.begin(), blocks.end()), blocks.end());
+      std::vector<int64_t> keys;
+      for (int64_t i : blocks)
+        for (int64_t j = i * c->C; j < std::min((i + 1) * c->C, c->N); ++j)
+          if (!c->causal || j <= t) keys.push_back(j);
+      if (keys.empty()) continue;
+      for (int64_t g = 0; g < G; ++g) {
+        const int64_t hq = h * G + g;
+        std::vector<double> qv(d), go(d), o(d, 0.0);
+        for (int64_t e = 0; e < d; ++e) {
+          qv[e] = elem(q, q_index(*c, b, hq, t, e), c->dtype);
+          go[e] = elem(dout, q_index(*c, b, hq, t, e), c->dtype);
+        }
+        std::vector<double> logit(keys.size());
+        for (size_t n2 = 0; n2 < keys.size(); ++n2) {
+          double s = 0;
+          for (int64_t e = 0; e < d; ++e) s += qv[e] * elem(k, kv_index(*c, b, h, keys[n2], e), c->dtype);
+          logit[n2] = sc * s;
+        }
+        const double z = logsumexp(logit);
+        std::vector<double> P(keys.size()), dP(keys.size());
+        for (size_t n2 = 0; n2 < keys.size(); ++n2) {
+          P[n2] = std::exp(logit[n2] - z);
+          double dp = 0;
+          for (int64_t e = 0; e < d; ++e) {
+            const double ve = elem(v, kv_index(*c, b, h, keys[n2], e), c->dtype);
+            o[e] += P[n2] * ve;
+            dp += go[e] * ve;
+          }
+          dP[n2] = dp;
+        }
+        double D = 0;
+        for (int64_t e = 0; e < d; ++e) D += go[e] * o[e];
+        double* dqr = dq + ((b * c->H_q + hq) * c->N + t) * d;
+        for (size_t n2 = 0; n2 < keys.size(); ++n2) {
+          const double dS = P[n2] * (dP[n2] - D);
+          double* dkr = dk + (bh * c->N + keys[n2]) * d;
+          double* dvr = dv + (bh * c->N + keys[n2]) * d;
+          for (int64_t e = 0; e < d; ++e) {
+            dqr[e] += sc * dS * elem(k, kv_index(*c, b, h, keys[n2], e), c->dtype);
+            dkr[e] += sc * dS * qv[e];
+            dvr[e] += P[n2] * go[e];
+          }
+        }
+      }
+    }
+  }
+}
+
 // Decode cache update (§Kernels, decoding paragraph: cache the mean pyramid
 // and, per new token, update only the current leaf mean and its ancestor
 // path). seq_keys: [n + 1, d] keys of one sequence and head, the new key last

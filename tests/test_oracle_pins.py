@@ -451,6 +451,56 @@ def test_exact_selector_finds_planted_needles(oracle):
     assert all(j in list(s) for s, j in zip(sel, want))
 
 
+# --------------------------------------------------------------- backward
+
+def _random_selection(w, rng):
+    """A valid selection [B, H_kv, N, K]: up to K distinct usable leaves per
+    row (some rows get fewer), ascending, -1 padded."""
+    M1 = -(-w.N // w.C)
+    sel = np.full((w.B, w.H_kv, w.N, w.K), -1, np.int32)
+    for b in range(w.B):
+        for h in range(w.H_kv):
+            for t in range(w.N):
+                nv = (t // w.C + 1) if w.causal else M1
+                m = int(rng.integers(1, min(w.K, nv) + 1))
+                sel[b, h, t, :m] = np.sort(rng.choice(nv, m, replace=False))
+    return sel
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_backward_matches_autograd(oracle, causal):
+    # Gradient of §BSA's attention over a fixed selection: torch autograd
+    # (fp64) through dense attention whose mask admits exactly the selected
+    # blocks' keys (and, causally, keys <= t); the GQA key/value sharing is a
+    # repeat over the group, so autograd sums the group's contributions.
+    w = _small(N=200, C=16, K=3, causal=causal, H_q=6, H_kv=2, d=16, seed=21)
+    x = workloads.prefill_inputs(w)
+    rng = np.random.default_rng(3)
+    sel = _random_selection(w, rng)
+    g = torch.randn(w.B, w.H_q, w.N, w.d, generator=torch.Generator().manual_seed(4))
+    dq, dk, dv = oracle.attn_bwd(_cfg(oracle, w), x["q"], x["k"], x["v"], sel, g)
+    G = w.H_q // w.H_kv
+    q = x["q"].double().requires_grad_()
+    k = x["k"].double().requires_grad_()
+    v = x["v"].double().requires_grad_()
+    allowed = torch.zeros(w.B, w.H_kv, w.N, w.N, dtype=torch.bool)
+    for b in range(w.B):
+        for h in range(w.H_kv):
+            for t in range(w.N):
+                for i in sel[b, h, t]:
+                    if i >= 0:
+                        allowed[b, h, t, i * w.C:(i + 1) * w.C] = True
+    if causal:
+        allowed &= torch.ones(w.N, w.N, dtype=torch.bool).tril()
+    mask = allowed.repeat_interleave(G, dim=1)
+    s = (q @ k.repeat_interleave(G, 1).transpose(-1, -2)) / math.sqrt(w.d)
+    p = torch.softmax(s.masked_fill(~mask, -math.inf), dim=-1)
+    o = p @ v.repeat_interleave(G, 1)
+    (o * g.double()).sum().backward()
+    for got, want in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
+        assert np.abs(got - want.numpy()).max() < 1e-10
+
+
 # ------------------------------------------------------------------ decode
 
 def test_decode_incremental_pyramid_equals_batch(oracle):
