@@ -369,6 +369,21 @@ def run_gpu(args):
     if needles:
         needles["flat"] = needle_recall(p.sel, x["needles"])
 
+    # Attention backward over the step's selection (training), once after a
+    # warm-up: dq, dk, dv (fp32) for a random output gradient.
+    bwd_ms = None
+    if w.dtype == "bf16":
+        p(q, k, v)
+        dout = torch.randn(q.shape, generator=torch.Generator(device=dev).manual_seed(11), device=dev).to(q.dtype)
+        api.sparse_attn_bwd(q, k, v, p.sel, p.out, p.lse, dout, C=w.C, causal=w.causal)
+        be0, be1 = events(2)
+        be0.record(stream)
+        grads = api.sparse_attn_bwd(q, k, v, p.sel, p.out, p.lse, dout, C=w.C, causal=w.causal)
+        be1.record(stream)
+        torch.cuda.synchronize()
+        bwd_ms = be0.elapsed_time(be1)
+        del grads, dout
+
     # End to end through the public API from pinned host buffers.
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     hout = torch.empty(p.out.shape, dtype=p.out.dtype).pin_memory()
@@ -421,6 +436,7 @@ def run_gpu(args):
         "select_speedup_vs_exact": exact_ms / stage_ms["select"] if stage_ms["select"] > 0 else None,
         "pisa_recall_vs_exact": recall,
         "needle_recall": needles,
+        "attn_bwd_ms": bwd_ms,
         "decode": decode,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

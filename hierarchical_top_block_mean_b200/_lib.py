@@ -53,6 +53,8 @@ SIGNATURES = {
     "pisa_select": (_i32, [_PC, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
     "pisa_select_flat": (_i32, [_PC, _p, _p, _p, _p]),
     "pisa_select_exact": (_i32, [_PC, _p, _p, _p, _p]),
+    "pisa_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_PC]),
+    "pisa_sparse_attn_bwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
     "pisa_sparse_attn_fwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p]),
     "pisa_select_noalloc": (_i32, [_PC, _p, _p, _p, _p, _p, _p]),
     "pisa_decode_pyramid_rows": (_i64, [_PD]),

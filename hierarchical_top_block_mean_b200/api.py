@@ -138,6 +138,26 @@ def select_flat(q, pyr, *, C: int, K: int, causal: bool, H_kv: int, scale: float
     return out
 
 
+def sparse_attn_bwd(q, k, v, sel, out, lse, dout, *, C: int, causal: bool, scale: float = 0.0):
+    """Gradients (dq, dk, dv; fp32) of the block-sparse attention with the
+    selection sel held fixed, for the output gradient dout; out and lse are the
+    forward's outputs. bf16 inputs."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, n, q.dtype)
+    _need(sel, "sel", torch.int32)
+    _need(lse, "lse", torch.float32)
+    pr = Problem.of(q, k, C=C, K=sel.shape[-1], causal=causal, scale=scale)
+    cfg = pr.cstruct()
+    nbytes = int(_lib.lib().pisa_attn_bwd_workspace_bytes(ctypes.byref(cfg)))
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    _lib.call("pisa_sparse_attn_bwd", ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(out), _p(lse), _p(dout),
+              _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(q))
+    return dq, dk, dv
+
+
 def select_exact(q, k, *, C: int, K: int, causal: bool, scale: float = 0.0, out=None):
     """Exact-score flat top-K: every usable leaf scored by its raw-key LSE
     summed over the group. sel [B, H_kv, N, K] int32."""

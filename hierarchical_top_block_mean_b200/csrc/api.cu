@@ -174,6 +174,26 @@ pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const vo
   return from_cuda(launch_attn_rows(args_of(cfg), q, k, v, sel, out, lse, as_stream(stream)));
 }
 
+size_t pisa_attn_bwd_workspace_bytes(const pisa_config* cfg) {
+  if (check_cfg(cfg) != PISA_OK) return 0;
+  return attn_bwd_workspace_bytes(args_of(cfg));
+}
+
+pisa_status pisa_sparse_attn_bwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
+                                 const int32_t* sel, const void* out, const float* lse, const void* dout, float* dq,
+                                 float* dk, float* dv, void* ws, size_t ws_bytes, void* stream) {
+  pisa_status s = check_cfg(cfg);
+  if (s != PISA_OK) return s;
+  if (cfg->dtype != PISA_DTYPE_BF16) return PISA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !sel || !out || !lse || !dout || !dq || !dk || !dv) return PISA_ERR_INVALID_ARGUMENT;
+  for (const void* p : {q, k, v, out, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                        static_cast<const void*>(dv)})
+    if (!aligned16(p)) return PISA_ERR_INVALID_ARGUMENT;
+  const PrefillArgs a = args_of(cfg);
+  if (!ws || !aligned16(ws) || ws_bytes < attn_bwd_workspace_bytes(a)) return PISA_ERR_WORKSPACE;
+  return from_cuda(launch_attn_bwd(a, q, k, v, sel, out, lse, dout, dq, dk, dv, ws, as_stream(stream)));
+}
+
 int64_t pisa_decode_pyramid_rows(const pisa_decode_config* cfg) {
   if (check_dcfg(cfg) != PISA_OK) return 0;
   return make_layout(cfg->cap, cfg->C).R;

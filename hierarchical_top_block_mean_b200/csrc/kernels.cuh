@@ -43,6 +43,12 @@ cudaError_t launch_decode_rows(const DecodeArgs& a, const Layout& lay, int mode,
                                const void* k_cache, const void* v_cache, const float* pyr, const int32_t* len,
                                int32_t* sel, void* out, float* lse, cudaStream_t st);
 
+// ---- attention backward over a fixed selection (bf16 inputs, fp32 gradients)
+size_t attn_bwd_workspace_bytes(const PrefillArgs& a);
+cudaError_t launch_attn_bwd(const PrefillArgs& a, const void* q, const void* k, const void* v, const int32_t* sel,
+                            const void* out, const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                            void* ws, cudaStream_t st);
+
 // ---- exact-score flat selection (every usable leaf scored by its raw-key LSE)
 cudaError_t launch_exact_rows(const PrefillArgs& a, const void* q, const void* k, int32_t* sel, cudaStream_t st);
 bool exact_umma_supported(const PrefillArgs& a);

@@ -196,6 +196,28 @@ pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const vo
 pisa_status pisa_select_noalloc(const pisa_config* cfg, const void* q, const void* k, const float* pyr, int32_t* sel,
                                 float* sel_score, void* stream);
 
+/*
+ * Backward of the block-sparse attention over a fixed selection — the
+ * gradient of pisa_sparse_attn_fwd with sel held constant (the selection is a
+ * discrete choice; only the attention over the selected blocks' keys is
+ * differentiated, §BSA). For a row (kv head, t) and a query head of the group,
+ * over the usable keys j of the selected blocks (causal: j <= t):
+ *   P_j = exp(scale q.k_j - lse), dP_j = dout.v_j, D = dout.out,
+ *   dS_j = P_j (dP_j - D); dq = scale sum_j dS_j k_j,
+ *   dk_j += scale dS_j q, dv_j += P_j dout (summed over rows and heads).
+ *   q, out, dout : [B, H_q, N, d] bf16 (out and lse as the forward wrote them);
+ *   k, v : [B, H_kv, N, d] bf16;  sel : [B, H_kv, N, K];  lse : [B, H_q, N];
+ *   dq : [B, H_q, N, d] fp32;  dk, dv : [B, H_kv, N, d] fp32 (overwritten).
+ * bf16 only (PISA_ERR_UNSUPPORTED otherwise). ws: at least
+ * pisa_attn_bwd_workspace_bytes(cfg) bytes, 16-byte aligned, else
+ * PISA_ERR_WORKSPACE. dk and dv are accumulated with atomics, so they are
+ * reproducible only up to fp32 rounding order.
+ */
+size_t pisa_attn_bwd_workspace_bytes(const pisa_config* cfg);
+pisa_status pisa_sparse_attn_bwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
+                                 const int32_t* sel, const void* out, const float* lse, const void* dout, float* dq,
+                                 float* dk, float* dv, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- decode
  * §Kernels, decoding: the mean pyramid is cached; per new token only the
  * current leaf mean and its ancestor path are updated, and one fused kernel
