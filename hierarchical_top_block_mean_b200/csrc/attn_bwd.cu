@@ -363,15 +363,22 @@ struct DkvSmem {
   static constexpr int kRows = 16;                        // (query, head) rows per query tile
   static constexpr int kK = 0;                            // K tile [CC][D]
   static constexpr int kV = kK + CC * D * 2;              // V tile [CC][D]
-  static constexpr int kQ = kV + CC * D * 2;              // Q rows [16][D]
-  static constexpr int kG = kQ + kRows * D * 2;           // dout rows [16][D]
-  static constexpr int kP = kG + kRows * D * 2;           // P [16][CC]
+  static constexpr int kQ = kV + CC * D * 2;              // Q rows [2][16][D] (double buffered)
+  static constexpr int kG = kQ + 2 * kRows * D * 2;       // dout rows [2][16][D]
+  static constexpr int kP = kG + 2 * kRows * D * 2;       // P [16][CC]
   static constexpr int kS = kP + kRows * CC * 2;          // dS [16][CC]
-  static constexpr int kL = kS + kRows * CC * 2;          // lse [16]
-  static constexpr int kDD = kL + kRows * 4;              // D [16]
-  static constexpr int kT = kDD + kRows * 4;              // query position per row [16]
-  static constexpr int kBytes = kT + kRows * 4 + 128;
+  static constexpr int kL = kS + kRows * CC * 2;          // lse [2][16]
+  static constexpr int kDD = kL + 2 * kRows * 4;          // D [2][16]
+  static constexpr int kT = kDD + 2 * kRows * 4;          // query position per row [2][16]
+  static constexpr int kTq = kT + 2 * kRows * 4;          // the item's query positions [kBwdPairs]
+  static constexpr int kBytes = kTq + kBwdPairs * 4 + 128;
 };
+
+// 4-byte asynchronous copy global -> shared; src_bytes = 0 writes zero.
+__device__ inline void cp_async4(void* smem, const void* gmem, int src_bytes) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(gmem), "r"(src_bytes));
+}
 
 template <int D, int CC, int G>
 __global__ void __launch_bounds__(kDkvWarps * 32)
@@ -394,6 +401,7 @@ __global__ void __launch_bounds__(kDkvWarps * 32)
   float* Ls = reinterpret_cast<float*>(sm + SM::kL);
   float* DDs = reinterpret_cast<float*>(sm + SM::kDD);
   int* Ts = reinterpret_cast<int*>(sm + SM::kT);
+  int* Tq = reinterpret_cast<int*>(sm + SM::kTq);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int64_t n = a.N;
@@ -407,6 +415,9 @@ __global__ void __launch_bounds__(kDkvWarps * 32)
     const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
     const int key_base = blk * CC;
     const int nkeys = static_cast<int>(min(static_cast<int64_t>(CC), n - key_base));
+    const int npairs = it.z - it.y;
+    const int ntiles = (npairs + kQT - 1) / kQT;
+    if (threadIdx.x < kBwdPairs) Tq[threadIdx.x] = threadIdx.x < npairs ? qlist[it.y + threadIdx.x] : -1;
     // The leaf's K and V rows (zero past the sequence).
     for (int i = threadIdx.x; i < CC * (D / 8); i += blockDim.x) {
       const int r = i / (D / 8), c = (i % (D / 8)) * 8;
@@ -415,36 +426,42 @@ __global__ void __launch_bounds__(kDkvWarps * 32)
       cp_async16(Ks + tsw<D>(r, c), k + src, ok ? 16 : 0);
       cp_async16(Vs + tsw<D>(r, c), v + src, ok ? 16 : 0);
     }
+    cp_async_commit();
+    __syncthreads();  // Tq
+    // Query tile i -> buffer f: rows r = (query qi, head g), qi = r / G.
+    auto issue = [&](int i, int f) {
+      for (int x = threadIdx.x; x < 16 * (D / 8); x += blockDim.x) {
+        const int r = x / (D / 8), c = (x % (D / 8)) * 8;
+        const int t = Tq[i * kQT + r / G];
+        const int64_t src = ((b * a.H_q + h * G + r % G) * n + (t >= 0 ? t : 0)) * D + c;
+        cp_async16(Qs + f * (16 * D * 2) + tsw<D>(r, c), q + src, t >= 0 ? 16 : 0);
+        cp_async16(Gs + f * (16 * D * 2) + tsw<D>(r, c), dout + src, t >= 0 ? 16 : 0);
+      }
+      if (threadIdx.x < 16) {
+        const int r = threadIdx.x;
+        const int t = Tq[i * kQT + r / G];
+        const int64_t lrow = (b * a.H_q + h * G + r % G) * n + (t >= 0 ? t : 0);
+        cp_async4(Ls + 16 * f + r, lse + lrow, t >= 0 ? 4 : 0);
+        cp_async4(DDs + 16 * f + r, Dv + lrow, t >= 0 ? 4 : 0);
+        Ts[16 * f + r] = t;
+      }
+    };
+    issue(0, 0);
+    cp_async_commit();
     float dka[kNT][4], dva[kNT][4];
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) dka[nt][i] = dva[nt][i] = 0.f;
 
-    for (int p0 = it.y; p0 < it.z; p0 += kQT) {
-      const int nq = min(kQT, it.z - p0);
-      // Query tile: rows r = (query qi, head g), qi = r / G.
-      for (int i = threadIdx.x; i < 16 * (D / 8); i += blockDim.x) {
-        const int r = i / (D / 8), c = (i % (D / 8)) * 8;
-        const int qi = r / G, g = r % G;
-        const bool ok = qi < nq;
-        const int t = ok ? qlist[p0 + qi] : 0;
-        const int64_t src = ((b * a.H_q + h * G + g) * n + t) * D + c;
-        cp_async16(Qs + tsw<D>(r, c), q + src, ok ? 16 : 0);
-        cp_async16(Gs + tsw<D>(r, c), dout + src, ok ? 16 : 0);
-      }
+    for (int i = 0; i < ntiles; ++i) {
+      const int f = i & 1;
+      if (i + 1 < ntiles) issue(i + 1, f ^ 1);
       cp_async_commit();
-      if (threadIdx.x < 16) {
-        const int r = threadIdx.x, qi = r / G, g = r % G;
-        const bool ok = qi < nq;
-        const int t = ok ? qlist[p0 + qi] : 0;
-        const int64_t lrow = (b * a.H_q + h * G + g) * n + t;
-        Ls[r] = ok ? lse[lrow] : 0.f;
-        DDs[r] = ok ? Dv[lrow] : 0.f;
-        Ts[r] = ok ? t : -1;
-      }
-      cp_async_wait<0>();
+      cp_async_wait<1>();  // K, V and tile i have landed
       __syncthreads();
+      const unsigned char* Qf = Qs + f * (16 * D * 2);
+      const unsigned char* Gf = Gs + f * (16 * D * 2);
 
       // Phase A: warp w < kNT takes keys [8 w, 8 w + 8): S = Q K^T and
       // dP = dO V^T over d, then P and dS into shared memory.
@@ -461,8 +478,8 @@ __global__ void __launch_bounds__(kDkvWarps * 32)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             uint32_t aq[4], ag[4];
-            ldsm_x4(aq, Qs + tsw<D>(arow, 16 * (ks + u) + 8 * (mi >> 1)));
-            ldsm_x4(ag, Gs + tsw<D>(arow, 16 * (ks + u) + 8 * (mi >> 1)));
+            ldsm_x4(aq, Qf + tsw<D>(arow, 16 * (ks + u) + 8 * (mi >> 1)));
+            ldsm_x4(ag, Gf + tsw<D>(arow, 16 * (ks + u) + 8 * (mi >> 1)));
             mma_bf16(s, aq, bk[2 * u], bk[2 * u + 1]);
             mma_bf16(dp, ag, bv[2 * u], bv[2 * u + 1]);
           }
@@ -470,8 +487,8 @@ __global__ void __launch_bounds__(kDkvWarps * 32)
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           const int r = gid + 8 * rr;
-          const int t = Ts[r];
-          const float l = Ls[r], dd = DDs[r];
+          const int t = Ts[16 * f + r];
+          const float l = Ls[16 * f + r], dd = DDs[16 * f + r];
           float pv[2], sv[2];
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
@@ -494,8 +511,8 @@ __global__ void __launch_bounds__(kDkvWarps * 32)
         uint32_t ag[4], aq[4];
         {
           const int r = (lane & 7) + 8 * (mi >> 1);
-          ldsm_x4_t(ag, Gs + tsw<D>(r, 16 * warp + 8 * (mi & 1)));
-          ldsm_x4_t(aq, Qs + tsw<D>(r, 16 * warp + 8 * (mi & 1)));
+          ldsm_x4_t(ag, Gf + tsw<D>(r, 16 * warp + 8 * (mi & 1)));
+          ldsm_x4_t(aq, Qf + tsw<D>(r, 16 * warp + 8 * (mi & 1)));
         }
         const int brow = (lane & 7) + 8 * (mi & 1);
 #pragma unroll
@@ -511,8 +528,9 @@ __global__ void __launch_bounds__(kDkvWarps * 32)
           }
         }
       }
-      __syncthreads();  // the next query tile overwrites Q, dO, P and dS
+      __syncthreads();  // P, dS and this buffer are rewritten two steps on
     }
+    cp_async_wait<0>();
     // The item's partial gradients: dV^T, dK^T rows d = 16 w + gid (+8),
     // columns keys 8 nt + 2 tig (+1).
     if (warp < kKS) {
@@ -529,7 +547,7 @@ __global__ void __launch_bounds__(kDkvWarps * 32)
           }
         }
     }
-    __syncthreads();  // K and V tiles are reloaded for the next item
+    __syncthreads();  // K, V and Tq are reloaded for the next item
   }
 }
 
