@@ -294,6 +294,45 @@ def time_decode(wd, steps=32, warmup=4):
     return {"workload": wd.name, "us_per_step": us, "select_us": us_sel, "steps": steps, "status_ok": ok}
 
 
+def time_decode_paged(wd, steps=32, warmup=4):
+    """µs per fused decode step over paged caches: the same workload with each
+    sequence's leaf blocks in pages of a shuffled pool (one leaf per page)."""
+    dev = torch.device("cuda")
+    kc, vc, lens = workloads.decode_cache(wd, device=dev)
+    max_pages = wd.cap // wd.C
+    perm = torch.randperm(wd.S * max_pages, generator=torch.Generator().manual_seed(1)).to(dev)
+
+    def pages(x):
+        y = x.reshape(wd.S, wd.H_kv, max_pages, wd.C, wd.d).permute(0, 2, 1, 3, 4).reshape(-1, wd.H_kv, wd.C, wd.d)
+        out = torch.empty_like(y)
+        out[perm] = y  # logical page i of the pool goes to physical page perm[i]
+        return out
+
+    kp = pages(kc)
+    del kc
+    vp = pages(vc)
+    del vc
+    bt = perm.reshape(wd.S, max_pages).to(torch.int32).contiguous()
+    st = api.PagedDecodeState(S=wd.S, max_pages=max_pages, H_q=wd.H_q, H_kv=wd.H_kv, d=wd.d, C=wd.C, K=wd.K,
+                              k_pages=kp, v_pages=vp, block_table=bt, lens=lens, dtype=wd.torch_dtype)
+    st.init()
+    ins = [workloads.decode_step_inputs(wd, s, device=dev) for s in range(steps + warmup)]
+    for s in range(warmup):
+        st.step(*ins[s], keep_sel=False)
+    e0, e1 = events(2)
+    torch.cuda.synchronize()
+    e0.record()
+    for s in range(warmup, warmup + steps):
+        st.step(*ins[s], keep_sel=False)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / steps
+    ok = int(st.status.item()) == 0
+    del st, kp, vp
+    torch.cuda.empty_cache()
+    return {"workload": wd.name + " (paged)", "us_per_step": us, "steps": steps, "status_ok": ok}
+
+
 def run_gpu(args):
     dist = dist_init(args.gpus)
     rank = dist.get_rank() if dist else 0
@@ -410,6 +449,7 @@ def run_gpu(args):
         del x
         torch.cuda.empty_cache()
         decode = time_decode(workloads.DECODE[args.decode_workload])
+        decode["paged"] = time_decode_paged(workloads.DECODE[args.decode_workload])
 
     pk, pk_kind = peaks()
     # Roofline of the dominant stage (the attention kernel: one launch per step).

@@ -64,6 +64,8 @@ SIGNATURES = {
     "pisa_decode_select": (_i32, [_PD, _p, _p, _p, _p, _p, _p]),
     "pisa_decode_attn": (_i32, [_PD, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
     "pisa_decode_step": (_i32, [_PD, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "pisa_decode_init_paged": (_i32, [_PD, _p, _p, ctypes.c_int, _p, _p, _p]),
+    "pisa_decode_step_paged": (_i32, [_PD, _p, _p, _p, _p, _p, _p, ctypes.c_int, _p, _p, _p, _p, _p, _p, _p, _p]),
 }
 
 _lock = threading.Lock()

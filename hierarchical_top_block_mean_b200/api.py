@@ -288,5 +288,51 @@ class DecodeState:
         return pyramid_geometry(self.cap, self.C)[1]
 
 
+class PagedDecodeState:
+    """Decode state over paged KV caches: k_pages / v_pages [num_pages, H_kv,
+    C, d], one leaf block of one sequence per page, and a block table
+    [S, max_pages] (int32, -1 for unassigned) mapping each sequence's leaves to
+    pages. The pyramid, lengths, status word and workspace are as in
+    DecodeState; capacity is max_pages * C tokens per sequence."""
+
+    def __init__(self, *, S: int, max_pages: int, H_q: int, H_kv: int, d: int, C: int, K: int, k_pages, v_pages,
+                 block_table, lens, dtype=torch.bfloat16, scale: float = 0.0):
+        dev = k_pages.device
+        cap = max_pages * C
+        self.cfg = _lib.DecodeConfig(S, cap, H_q, H_kv, d, C, 2, K, _DT[dtype], scale)
+        self.S, self.cap, self.max_pages, self.H_q, self.H_kv, self.d, self.C, self.K = S, cap, max_pages, H_q, H_kv, d, C, K
+        for t, n in ((k_pages, "k_pages"), (v_pages, "v_pages")):
+            _need(t, n, dtype)
+        _need(block_table, "block_table", torch.int32)
+        _need(lens, "lens", torch.int32)
+        if tuple(block_table.shape) != (S, max_pages):
+            raise ValueError("block_table must be [S, max_pages]")
+        self.k_pages, self.v_pages, self.block_table, self.len = k_pages, v_pages, block_table, lens
+        R = int(_lib.lib().pisa_decode_pyramid_rows(ctypes.byref(self.cfg)))
+        if R <= 0:
+            raise _lib.PisaError("pisa_decode_pyramid_rows", 1)
+        self.R = R
+        self.pyr = torch.zeros((S, H_kv, R, d), dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.sel = torch.empty((S, H_kv, K), dtype=torch.int32, device=dev)
+        self.out = torch.empty((S, H_q, d), dtype=dtype, device=dev)
+        self.lse = torch.empty((S, H_q), dtype=torch.float32, device=dev)
+        ws = int(_lib.lib().pisa_decode_workspace_bytes(ctypes.byref(self.cfg)))
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+
+    def init(self):
+        """Builds each sequence's pyramid over its first len[s] cached tokens."""
+        _lib.call("pisa_decode_init_paged", ctypes.byref(self.cfg), _p(self.k_pages), _p(self.block_table),
+                  self.max_pages, _p(self.pyr), _p(self.len), _stream(self.pyr))
+
+    def step(self, q_new, k_new, v_new, keep_sel: bool = True):
+        """Append + select + attend for every sequence."""
+        _lib.call("pisa_decode_step_paged", ctypes.byref(self.cfg), _p(q_new), _p(k_new), _p(v_new),
+                  _p(self.k_pages), _p(self.v_pages), _p(self.block_table), self.max_pages, _p(self.pyr),
+                  _p(self.len), _p(self.sel) if keep_sel else None, _p(self.out), _p(self.lse), _p(self.status),
+                  _p(self.workspace), _stream(self.pyr))
+        return self.out
+
+
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)

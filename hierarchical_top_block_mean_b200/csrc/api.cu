@@ -215,6 +215,46 @@ pisa_status pisa_decode_init(const pisa_decode_config* cfg, const void* k_cache,
                                         cfg->S * cfg->H_kv, cfg->H_kv, cfg->cap, cfg->C, as_stream(stream)));
 }
 
+namespace {
+// Paged caches: fused path only, one leaf block per page, cap = max_pages * C.
+pisa_status check_paged(const pisa_decode_config* cfg, const int32_t* block_table, int max_pages) {
+  pisa_status s = check_dcfg(cfg);
+  if (s != PISA_OK) return s;
+  if (!block_table || max_pages < 1 || static_cast<int64_t>(max_pages) * cfg->C != cfg->cap)
+    return PISA_ERR_INVALID_ARGUMENT;
+  if (!decode_fused_supported(dargs_of(cfg))) return PISA_ERR_UNSUPPORTED;
+  return PISA_OK;
+}
+}  // namespace
+
+pisa_status pisa_decode_init_paged(const pisa_decode_config* cfg, const void* k_pages, const int32_t* block_table,
+                                   int max_pages, float* pyr, const int32_t* len, void* stream) {
+  pisa_status s = check_paged(cfg, block_table, max_pages);
+  if (s != PISA_OK) return s;
+  if (!k_pages || !pyr || !len || !aligned16(k_pages) || !aligned16(pyr)) return PISA_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(cfg->cap, cfg->C);
+  return from_cuda(launch_build_pyramid(cfg->dtype, cfg->d, k_pages, pyr, lay, cfg->cap, 0, len,
+                                        cfg->S * cfg->H_kv, cfg->H_kv, cfg->cap, cfg->C, as_stream(stream),
+                                        PageMap{block_table, max_pages}));
+}
+
+pisa_status pisa_decode_step_paged(const pisa_decode_config* cfg, const void* q_new, const void* k_new,
+                                   const void* v_new, void* k_pages, void* v_pages, const int32_t* block_table,
+                                   int max_pages, float* pyr, int32_t* len, int32_t* sel, void* out, float* lse,
+                                   int32_t* status, void* workspace, void* stream) {
+  pisa_status s = check_paged(cfg, block_table, max_pages);
+  if (s != PISA_OK) return s;
+  if (!q_new || !k_new || !v_new || !k_pages || !v_pages || !pyr || !len || !out || !status)
+    return PISA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q_new) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(pyr))
+    return PISA_ERR_INVALID_ARGUMENT;
+  if (!workspace || !aligned16(workspace)) return PISA_ERR_WORKSPACE;
+  const Layout lay = make_layout(cfg->cap, cfg->C);
+  return from_cuda(launch_decode_fused(dargs_of(cfg), lay, 7, q_new, k_new, v_new, k_pages, v_pages, pyr, len, sel,
+                                       out, lse, status, static_cast<float*>(workspace), as_stream(stream),
+                                       block_table, max_pages));
+}
+
 pisa_status pisa_decode_append(const pisa_decode_config* cfg, const void* k_new, const void* v_new, void* k_cache,
                                void* v_cache, float* pyr, int32_t* len, int32_t* status, void* stream) {
   pisa_status s = check_dcfg(cfg);

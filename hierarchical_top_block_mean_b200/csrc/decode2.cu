@@ -153,13 +153,13 @@ __device__ inline void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
 }
 
-template <int D, int CC, int G>
+template <int D, int CC, int G, bool PAGED>
 __global__ void __launch_bounds__(kDecWarps * 32, 4)
     decode_kernel(DecodeArgs a, Layout lay, int mode, const bf16* __restrict__ q_new, const bf16* __restrict__ k_new,
                   const bf16* __restrict__ v_new, bf16* __restrict__ kc, bf16* __restrict__ vc,
                   float* __restrict__ pyr, int32_t* __restrict__ len, int32_t* __restrict__ sel,
                   bf16* __restrict__ out, float* __restrict__ lse, int32_t* __restrict__ status,
-                  float* lgt_ws) {
+                  float* lgt_ws, const int32_t* __restrict__ bt, int max_pages) {
   using LM = LeafMean<bf16, D>;
   using SM = DecSmem<D, CC, G>;
   constexpr int kKS = D / 16, kMT = CC / 16;
@@ -177,8 +177,17 @@ __global__ void __launch_bounds__(kDecWarps * 32, 4)
   const int64_t s = blockIdx.x / a.H_kv, h = blockIdx.x % a.H_kv;
   const int64_t bh = s * a.H_kv + h;
   const int C = a.C, K = a.K;
-  const bf16* kh = kc + bh * a.cap * D;
-  const bf16* vh = vc + bh * a.cap * D;
+  // Element offset of key (and value) row j of this (sequence, kv head):
+  // dense caches [S, H_kv, cap, D]; paged caches hold leaf j / C of the
+  // sequence in page bt[s][j / C], laid out [page][H_kv][C][D].
+  auto kv_row = [&](int64_t j) -> int64_t {
+    if constexpr (PAGED) {
+      const int64_t pg = bt[s * max_pages + j / CC];
+      return ((pg * a.H_kv + h) * CC + j % CC) * D;
+    } else {
+      return (bh * a.cap + j) * D;
+    }
+  };
   const int64_t n0 = len[s];
   int64_t nn = n0;
   if (mode & kModeAppend) {
@@ -186,10 +195,11 @@ __global__ void __launch_bounds__(kDecWarps * 32, 4)
     // its existing keys now.
     if (threadIdx.x == 0 && n0 > 0 && n0 < a.cap) {
       const int64_t lk0 = (n0 / C) * C;
-      if (n0 > lk0) prefetch_l2(kh + lk0 * D, static_cast<uint32_t>((n0 - lk0) * D * 2));
+      if (n0 > lk0) prefetch_l2(kc + kv_row(lk0), static_cast<uint32_t>((n0 - lk0) * D * 2));
     }
     cg::this_cluster().sync();  // every CTA of this sequence has read len[s]
-    if (n0 >= a.cap || n0 < 0) {
+    // Full: no room left, or (paged) no page for the new token's leaf.
+    if (n0 >= a.cap || n0 < 0 || (PAGED && bt[s * max_pages + n0 / CC] < 0)) {
       if (h == 0 && threadIdx.x == 0) *status = PISA_ERR_CAPACITY;
     } else {
       nn = n0 + 1;
@@ -214,12 +224,12 @@ __global__ void __launch_bounds__(kDecWarps * 32, 4)
     const int nold = static_cast<int>(n - lo);
     for (int i = threadIdx.x; i < nold * (D / 8); i += blockDim.x) {
       const int r = i / (D / 8), c8 = i % (D / 8);
-      cp_async16(lrows + r * D + c8 * 8, kh + (lo + r) * D + c8 * 8, 16);
+      cp_async16(lrows + r * D + c8 * 8, kc + kv_row(lo + r) + c8 * 8, 16);
     }
     cp_async_commit();
     if (warp == 0) {
-      bf16* kr = kc + (bh * a.cap + n) * D;
-      bf16* vr = vc + (bh * a.cap + n) * D;
+      bf16* kr = kc + kv_row(n);
+      bf16* vr = vc + kv_row(n);
       for (int e = lane; e < D / 2; e += 32) {
         const uint32_t kw = reinterpret_cast<const uint32_t*>(k_new + bh * D)[e];
         reinterpret_cast<uint32_t*>(kr)[e] = kw;
@@ -351,7 +361,7 @@ __global__ void __launch_bounds__(kDecWarps * 32, 4)
                 [&](int u) -> TileSrc {
                   const int64_t k0 = static_cast<int64_t>(wc[warp + kDecWarps * (u / kMT)]) * CC + 16 * (u % kMT);
                   const int64_t nv = nn - k0;
-                  return nv > 0 ? TileSrc{kh + k0 * D, nv < 16 ? static_cast<int>(nv) : 16} : TileSrc{kh, 0};
+                  return nv > 0 ? TileSrc{kc + kv_row(k0), nv < 16 ? static_cast<int>(nv) : 16} : TileSrc{kc, 0};
                 },
                 [&](int u, const bf16* t) {
                   const int x = warp + kDecWarps * (u / kMT), mt = u % kMT;
@@ -443,7 +453,7 @@ __global__ void __launch_bounds__(kDecWarps * 32, 4)
           [&](int u) -> TileSrc {
             const int64_t k0 = static_cast<int64_t>(blk[warp + kDecWarps * (u / kMT)]) * CC + 16 * (u % kMT);
             const int64_t nv = nn - k0;
-            return nv > 0 ? TileSrc{kh + k0 * D, nv < 16 ? static_cast<int>(nv) : 16} : TileSrc{kh, 0};
+            return nv > 0 ? TileSrc{kc + kv_row(k0), nv < 16 ? static_cast<int>(nv) : 16} : TileSrc{kc, 0};
           },
           [&](int u, const bf16* t) {
             const int x = warp + kDecWarps * (u / kMT);
@@ -461,7 +471,7 @@ __global__ void __launch_bounds__(kDecWarps * 32, 4)
         [&](int u) -> TileSrc {
           const int64_t k0 = static_cast<int64_t>(blk[warp + kDecWarps * (u / kMT)]) * CC + 16 * (u % kMT);
           const int64_t nv = nn - k0;
-          return nv > 0 ? TileSrc{vh + k0 * D, nv < 16 ? static_cast<int>(nv) : 16} : TileSrc{vh, 0};
+          return nv > 0 ? TileSrc{vc + kv_row(k0), nv < 16 ? static_cast<int>(nv) : 16} : TileSrc{vc, 0};
         },
         [&](int u, const bf16* t) {
           const int x = warp + kDecWarps * (u / kMT), kk = u % kMT;
@@ -574,10 +584,11 @@ int64_t decode_logit_floats(const DecodeArgs& a) {
 cudaError_t launch_decode_fused(const DecodeArgs& a, const Layout& lay, int mode, const void* q_new,
                                 const void* k_new, const void* v_new, void* k_cache, void* v_cache, float* pyr,
                                 int32_t* len, int32_t* sel, void* out, float* lse, int32_t* status, float* lgt_ws,
-                                cudaStream_t st) {
+                                cudaStream_t st, const int32_t* block_table, int max_pages) {
   return dispatch_tdg(PISA_DTYPE_BF16, a.d, a.H_q / a.H_kv, [&](auto, auto dd, auto gg) -> cudaError_t {
     constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
-    auto kern = a.C == 64 ? decode_kernel<D, 64, G> : decode_kernel<D, 32, G>;
+    auto kern = block_table ? (a.C == 64 ? decode_kernel<D, 64, G, true> : decode_kernel<D, 32, G, true>)
+                            : (a.C == 64 ? decode_kernel<D, 64, G, false> : decode_kernel<D, 32, G, false>);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(a.S * a.H_kv));
     cfg.blockDim = dim3(kDecWarps * 32);
@@ -596,7 +607,7 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, const Layout& lay, int mode
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, lay, mode, static_cast<const bf16*>(q_new),
                                        static_cast<const bf16*>(k_new), static_cast<const bf16*>(v_new),
                                        static_cast<bf16*>(k_cache), static_cast<bf16*>(v_cache), pyr, len, sel,
-                                       static_cast<bf16*>(out), lse, status, lgt_ws);
+                                       static_cast<bf16*>(out), lse, status, lgt_ws, block_table, max_pages);
     count_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

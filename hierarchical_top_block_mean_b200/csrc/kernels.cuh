@@ -55,12 +55,14 @@ bool exact_umma_supported(const PrefillArgs& a);
 cudaError_t launch_exact_umma(const PrefillArgs& a, const void* q, const void* k, int32_t* sel, cudaStream_t st);
 
 // Fused decode (bf16, H_kv <= 8, G_Q <= 8). mode bits: 1 append, 2 select, 4 attend.
-// lgt_ws: decode_logit_floats(a) floats, required when attending.
+// lgt_ws: decode_logit_floats(a) floats, required when attending. With a
+// block table the caches are pages [num_pages][H_kv][C][d], page
+// block_table[s * max_pages + i] holding leaf i of sequence s (cap = max_pages C).
 bool decode_fused_supported(const DecodeArgs& a);
 int64_t decode_logit_floats(const DecodeArgs& a);
 cudaError_t launch_decode_fused(const DecodeArgs& a, const Layout& lay, int mode, const void* q_new,
                                 const void* k_new, const void* v_new, void* k_cache, void* v_cache, float* pyr,
                                 int32_t* len, int32_t* sel, void* out, float* lse, int32_t* status, float* lgt_ws,
-                                cudaStream_t st);
+                                cudaStream_t st, const int32_t* block_table = nullptr, int max_pages = 0);
 
 }  // namespace pisa

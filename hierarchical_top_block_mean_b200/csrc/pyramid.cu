@@ -30,7 +30,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kLeafWarps * 32) pyramid_leaf_kernel(const T* __restrict__ k, float* __restrict__ pyr,
                                                                        Layout lay, int64_t n_uniform,
                                                                        const int32_t* __restrict__ len, int H,
-                                                                       int64_t k_rows, int C) {
+                                                                       int64_t k_rows, int C, PageMap pm) {
   __shared__ __align__(16) float sm[2][kLeafWarps][D];
   const int bh = blockIdx.y;
   const int b = bh / H;
@@ -47,7 +47,13 @@ __global__ void __launch_bounds__(kLeafWarps * 32) pyramid_leaf_kernel(const T* 
   const int64_t leaf = leaf0 + warp;
   if (leaf < M1) {
     float mean[LeafMean<T, D>::kVec];
-    leaf_mean_warp<T, D>(kbh, leaf * C, (leaf + 1) * C < n ? (leaf + 1) * C : n, mean);
+    const int64_t hi = (leaf + 1) * C < n ? (leaf + 1) * C : n;
+    if (pm.bt) {  // the leaf's keys are rows 0 .. of its page (same summation order)
+      const int64_t page = pm.bt[static_cast<int64_t>(b) * pm.max_pages + leaf];
+      leaf_mean_warp<T, D>(k + (page * H + bh % H) * C * D, 0, hi - leaf * C, mean);
+    } else {
+      leaf_mean_warp<T, D>(kbh, leaf * C, hi, mean);
+    }
     LeafMean<T, D>::store(mean, &sm[0][warp][0], pbh + (lay.off[1] + leaf) * D, lane);
   }
   // Levels above the leaves that lie inside this CTA's subtree.
@@ -114,11 +120,11 @@ __global__ void __launch_bounds__(256) pyramid_upper_kernel(float* __restrict__ 
 
 template <typename T, int D>
 cudaError_t build_impl(const void* k, float* pyr, const Layout& lay, int64_t n_max, int64_t n_uniform,
-                       const int32_t* len, int BH, int H, int64_t k_rows, int C, cudaStream_t st) {
+                       const int32_t* len, int BH, int H, int64_t k_rows, int C, PageMap pm, cudaStream_t st) {
   const int64_t M1 = level_size(n_max, C, 1);
   dim3 grid(static_cast<unsigned>((M1 + kLeafWarps - 1) / kLeafWarps), BH);
   pyramid_leaf_kernel<T, D><<<grid, kLeafWarps * 32, 0, st>>>(static_cast<const T*>(k), pyr, lay, n_uniform, len, H,
-                                                               k_rows, C);
+                                                               k_rows, C, pm);
   count_launch();
   cudaError_t err = cudaGetLastError();
   const int L = num_levels(n_max, C);
@@ -136,13 +142,13 @@ cudaError_t build_impl(const void* k, float* pyr, const Layout& lay, int64_t n_m
 
 cudaError_t launch_build_pyramid(int dtype, int D, const void* k, float* pyr, const Layout& lay, int64_t n_max,
                                  int64_t n_uniform, const int32_t* len, int BH, int H, int64_t k_rows, int C,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, PageMap pm) {
   if (dtype == PISA_DTYPE_BF16) {
-    if (D == 128) return build_impl<bf16, 128>(k, pyr, lay, n_max, n_uniform, len, BH, H, k_rows, C, st);
-    return build_impl<bf16, 64>(k, pyr, lay, n_max, n_uniform, len, BH, H, k_rows, C, st);
+    if (D == 128) return build_impl<bf16, 128>(k, pyr, lay, n_max, n_uniform, len, BH, H, k_rows, C, pm, st);
+    return build_impl<bf16, 64>(k, pyr, lay, n_max, n_uniform, len, BH, H, k_rows, C, pm, st);
   }
-  if (D == 128) return build_impl<float, 128>(k, pyr, lay, n_max, n_uniform, len, BH, H, k_rows, C, st);
-  return build_impl<float, 64>(k, pyr, lay, n_max, n_uniform, len, BH, H, k_rows, C, st);
+  if (D == 128) return build_impl<float, 128>(k, pyr, lay, n_max, n_uniform, len, BH, H, k_rows, C, pm, st);
+  return build_impl<float, 64>(k, pyr, lay, n_max, n_uniform, len, BH, H, k_rows, C, pm, st);
 }
 
 }  // namespace pisa

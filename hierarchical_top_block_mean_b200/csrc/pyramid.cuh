@@ -72,11 +72,19 @@ __device__ inline void leaf_mean_warp(const T* __restrict__ kbh, int64_t lo, int
   for (int e = 0; e < LM::kVec; ++e) mean[e] = acc[e] / cnt;
 }
 
+// Key rows held in pages: page bt[b * max_pages + i] holds the C keys of leaf
+// i of sequence b for every head, as [H][C][D] rows. bt == nullptr: dense
+// [B, H, k_rows, D] keys.
+struct PageMap {
+  const int32_t* bt;
+  int max_pages;
+};
+
 // Builds pyr for every (b, h) over its first n_b tokens (n_b = len[b] when len
 // is given, else n_uniform) into a layout sized for lay; k has k_rows rows per
 // head. n_max bounds every n_b.
 cudaError_t launch_build_pyramid(int dtype, int D, const void* k, float* pyr, const Layout& lay, int64_t n_max,
                                  int64_t n_uniform, const int32_t* len, int BH, int H, int64_t k_rows, int C,
-                                 cudaStream_t st);
+                                 cudaStream_t st, PageMap pm = PageMap{nullptr, 0});
 
 }  // namespace pisa

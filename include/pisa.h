@@ -271,6 +271,27 @@ pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, c
                              void* k_cache, void* v_cache, float* pyr, int32_t* len, int32_t* sel, void* out,
                              float* lse, int32_t* status, void* workspace, void* stream);
 
+/* ------------------------------------------------------ paged decode
+ * The same decode path over KV caches held in fixed-size pages, as serving
+ * systems keep them: one page holds one leaf block (C tokens) of one sequence
+ * for every kv head.
+ *   k_pages, v_pages : [num_pages, H_kv, C, d] in dtype (bf16 only);
+ *   block_table      : [S, max_pages] int32 device; entry i is the page of
+ *                      leaf i of the sequence, -1 where none is assigned;
+ *   cfg->cap         : must equal max_pages * C.
+ * Pages of the leaves a sequence already holds must be assigned. A step whose
+ * new token falls in a leaf without a page stores PISA_ERR_CAPACITY in status
+ * and skips that sequence, as a full dense cache does. Results are bit-for-bit
+ * those of the dense calls on the same data. Other arguments as for
+ * pisa_decode_init and pisa_decode_step; PISA_ERR_UNSUPPORTED when the
+ * configuration has no fused kernel (see pisa_decode_step). */
+pisa_status pisa_decode_init_paged(const pisa_decode_config* cfg, const void* k_pages, const int32_t* block_table,
+                                   int max_pages, float* pyr, const int32_t* len, void* stream);
+pisa_status pisa_decode_step_paged(const pisa_decode_config* cfg, const void* q_new, const void* k_new,
+                                   const void* v_new, void* k_pages, void* v_pages, const int32_t* block_table,
+                                   int max_pages, float* pyr, int32_t* len, int32_t* sel, void* out, float* lse,
+                                   int32_t* status, void* workspace, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
