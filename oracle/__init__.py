@@ -68,6 +68,8 @@ def _load():
             lib.oracle_select_flat_rows.argtypes = [ctypes.POINTER(Cfg), p, p, i64, p, p, p]
             lib.oracle_select_exact_rows.restype = None
             lib.oracle_attn_bwd.restype = None
+            lib.oracle_attn_bwd_dq_rows.restype = None
+            lib.oracle_attn_bwd_dq_rows.argtypes = [ctypes.POINTER(Cfg), p, p, p, i64, p, p, p, p]
             lib.oracle_attn_bwd.argtypes = [ctypes.POINTER(Cfg), p, p, p, p, p, p, p, p]
             lib.oracle_select_exact_rows.argtypes = [ctypes.POINTER(Cfg), p, p, i64, p, p, p]
             lib.oracle_attn_rows.restype = None
@@ -221,6 +223,23 @@ def attn_bwd(cfg: Cfg, q, k, v, sel, dout):
     _load().oracle_attn_bwd(ctypes.byref(cfg), _ptr(qa), _ptr(ka), _ptr(va), _ptr(s), _ptr(ga), _ptr(dq), _ptr(dk),
                             _ptr(dv))
     return dq, dk, dv
+
+
+def attn_bwd_dq_rows(cfg: Cfg, q, k, v, rows, sel, dout):
+    """dq of the attention backward for rows (b, kv head, t) only, given their
+    selections sel [n, K]: returns [n, G, d] fp64."""
+    qa, _ = _storage(q)
+    ka, _ = _storage(k)
+    va, _ = _storage(v)
+    ga, _ = _storage(dout)
+    r = _rows(rows)
+    n = r.shape[0]
+    G = cfg.H_q // cfg.H_kv
+    s = np.ascontiguousarray(np.asarray(sel, dtype=np.int32).reshape(n, cfg.K))
+    dq = np.zeros((n, G, cfg.d), np.float64)
+    _load().oracle_attn_bwd_dq_rows(ctypes.byref(cfg), _ptr(qa), _ptr(ka), _ptr(va), n, _ptr(r), _ptr(s), _ptr(ga),
+                                    _ptr(dq))
+    return dq
 
 
 def decode_append(seq_keys, n: int, C: int, cap: int, pyr: np.ndarray) -> None:

@@ -499,6 +499,64 @@ void oracle_attn_bwd(const oracle_cfg* c, const void* q, const void* k, const vo
   }
 }
 
+// dq of the attention backward for a list of rows only (a row's dq depends on
+// that row alone): the same formulas as oracle_attn_bwd, restricted to the
+// given (b, kv head, t) rows. sel: [n, K] the rows' selections; dout as q.
+// dq: [n, G, d].
+void oracle_attn_bwd_dq_rows(const oracle_cfg* c, const void* q, const void* k, const void* v, int64_t n,
+                             const int64_t* rows, const int32_t* sel, const void* dout, double* dq) {
+  const int64_t G = c->H_q / c->H_kv;
+  const double sc = cfg_scale(*c);
+  const int64_t d = c->d;
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t r = 0; r < n; ++r) {
+    const int64_t b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+    std::vector<int64_t> blocks;
+    for (int64_t m = 0; m < c->K; ++m)
+      if (sel[r * c->K + m] >= 0) blocks.push_back(sel[r * c->K + m]);
+    std::sort(blocks.begin(), blocks.end());
+    blocks.erase(std::unique(blocks.begin(), blocks.end()), blocks.end());
+    std::vector<int64_t> keys;
+    for (int64_t i : blocks)
+      for (int64_t j = i * c->C; j < std::min((i + 1) * c->C, c->N); ++j)
+        if (!c->causal || j <= t) keys.push_back(j);
+    for (int64_t g = 0; g < G; ++g) {
+      double* out = dq + (r * G + g) * d;
+      std::fill(out, out + d, 0.0);
+      if (keys.empty()) continue;
+      const int64_t hq = h * G + g;
+      std::vector<double> qv(d), go(d), o(d, 0.0);
+      for (int64_t e = 0; e < d; ++e) {
+        qv[e] = elem(q, q_index(*c, b, hq, t, e), c->dtype);
+        go[e] = elem(dout, q_index(*c, b, hq, t, e), c->dtype);
+      }
+      std::vector<double> logit(keys.size()), P(keys.size()), dP(keys.size());
+      for (size_t n2 = 0; n2 < keys.size(); ++n2) {
+        double s = 0;
+        for (int64_t e = 0; e < d; ++e) s += qv[e] * elem(k, kv_index(*c, b, h, keys[n2], e), c->dtype);
+        logit[n2] = sc * s;
+      }
+      const double z = logsumexp(logit);
+      for (size_t n2 = 0; n2 < keys.size(); ++n2) {
+        P[n2] = std::exp(logit[n2] - z);
+        double dp = 0;
+        for (int64_t e = 0; e < d; ++e) {
+          const double ve = elem(v, kv_index(*c, b, h, keys[n2], e), c->dtype);
+          o[e] += P[n2] * ve;
+          dp += go[e] * ve;
+        }
+        dP[n2] = dp;
+      }
+      double D = 0;
+      for (int64_t e = 0; e < d; ++e) D += go[e] * o[e];
+      for (size_t n2 = 0; n2 < keys.size(); ++n2) {
+        const double dS = P[n2] * (dP[n2] - D);
+        for (int64_t e = 0; e < d; ++e) out[e] += sc * dS * elem(k, kv_index(*c, b, h, keys[n2], e), c->dtype);
+      }
+    }
+  }
+}
+
 // Decode cache update (§Kernels, decoding paragraph: cache the mean pyramid
 // and, per new token, update only the current leaf mean and its ancestor
 // path). seq_keys: [n + 1, d] keys of one sequence and head, the new key last

@@ -501,6 +501,22 @@ def test_attention_backward_matches_autograd(oracle, causal):
         assert np.abs(got - want.numpy()).max() < 1e-10
 
 
+def test_attention_backward_dq_rows_match_all_rows(oracle):
+    # A row's dq depends on that row alone: the per-row entry point (used for
+    # sampled rows at full size) must reproduce the all-rows gradient.
+    w = _small(N=150, C=16, K=3, causal=True, H_q=4, H_kv=2, d=16, seed=23)
+    x = workloads.prefill_inputs(w)
+    sel = _random_selection(w, np.random.default_rng(5))
+    g = torch.randn(w.B, w.H_q, w.N, w.d, generator=torch.Generator().manual_seed(6))
+    dq, _, _ = oracle.attn_bwd(_cfg(oracle, w), x["q"], x["k"], x["v"], sel, g)
+    rows = [(0, h, t) for h in range(w.H_kv) for t in range(0, w.N, 7)]
+    got = oracle.attn_bwd_dq_rows(_cfg(oracle, w), x["q"], x["k"], x["v"], rows,
+                                  np.stack([sel[b, h, t] for (b, h, t) in rows]), g)
+    G = w.H_q // w.H_kv
+    for r, (b, h, t) in enumerate(rows):
+        assert np.abs(got[r] - dq[b, h * G:(h + 1) * G, t]).max() < 1e-12
+
+
 # ------------------------------------------------------------------ decode
 
 def test_decode_incremental_pyramid_equals_batch(oracle):

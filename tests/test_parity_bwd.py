@@ -67,3 +67,27 @@ def test_backward_rejects_fp32_and_small_workspace():
     lse = torch.zeros((w.B, w.H_q, w.N), dtype=torch.float32, device=dev)
     with pytest.raises(Exception):
         api.sparse_attn_bwd(q, k, v, sel, q, lse, q, C=w.C, causal=w.causal)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,rows", [("needle_16k", 256), ("needle_256k", 64)])
+def test_attention_backward_dq_full_size(name, rows):
+    # dk and dv gather every row that selects a block, out of reach of the
+    # oracle at full size; dq of a row depends on that row alone, so sampled
+    # rows are checked exactly as the small cases are.
+    w = workloads.PREFILL[name]
+    dev = torch.device("cuda")
+    x = workloads.prefill_inputs(w, device=dev)
+    q, k, v = x["q"], x["k"], x["v"]
+    p = api.Prefill(api.Problem.of(q, k, C=w.C, K=w.K, causal=w.causal), dev)
+    p(q, k, v)
+    dout = torch.randn(q.shape, generator=torch.Generator(device=dev).manual_seed(w.seed + 7), device=dev).to(q.dtype)
+    dq, _, _ = api.sparse_attn_bwd(q, k, v, p.sel, p.out, p.lse, dout, C=w.C, causal=w.causal)
+    torch.cuda.synchronize()
+    r = P.sample_rows(w, rows)
+    ref = O.attn_bwd_dq_rows(P.ocfg(w), P.host(q), P.host(k), P.host(v), r, P.gather_rows(p.sel, r), P.host(dout))
+    G = w.H_q // w.H_kv
+    d = P.host(dq).numpy()
+    hq = r[:, 1:2] * G + np.arange(G)[None, :]
+    got = d[r[:, 0:1], hq, r[:, 2:3], :]
+    print(name, _check(f"{name} dq", got, ref))
