@@ -176,24 +176,25 @@ __global__ void __launch_bounds__(kExThreads, 2)
       const int nv = qok ? static_cast<int>(lim < 0 ? 0 : (lim > 64 ? 64 : lim)) : 0;
       float u = 0.f;
       if (nv > 0) {
-        float mx = -INFINITY;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (nv >= 64) {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
+          for (int j = 0; j < 64; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
         } else {
 #pragma unroll
           for (int j = 0; j < 64; ++j)
-            if (j < nv) mx = fmaxf(mx, __uint_as_float(v[j]));
+            if (j < nv) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
         }
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         const float mxs = mx * sl2;
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
         if (nv >= 64) {
 #pragma unroll
-          for (int j = 0; j < 64; ++j) s4[j & 3] += exp2f(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+          for (int j = 0; j < 64; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
         } else {
 #pragma unroll
           for (int j = 0; j < 64; ++j)
-            if (j < nv) s4[j & 3] += exp2f(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+            if (j < nv) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
         }
         u = mx * a.scale + logf((s4[0] + s4[1]) + (s4[2] + s4[3]));
       }

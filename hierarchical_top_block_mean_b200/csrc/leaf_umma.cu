@@ -39,6 +39,7 @@ constexpr int kUmmaThreads = 32 * (kMmaWarp + 1);
 constexpr int kLoaders = 32 * kLoadWarps;
 constexpr int kTilePairs = 16;             // queries per MMA tile (x 8 heads = 128 rows)
 constexpr int kQStages = 5;
+constexpr int kLag = 2;                    // loader publishes a stage kLag tiles after filling it
 constexpr int kQStageBytes = kTilePairs * 8 * 128 * 2;  // 16 queries x 8 heads x 256 B = 32 KB (two 64-col halves)
 constexpr int kKeyBytes = 64 * 128 * 2;                 // 16 KB (two 64-col halves)
 constexpr int kAccCols = 64;                            // fp32 columns per accumulator (N = 64 keys)
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const int g0 = 2 * lw + (lane >> 4);          // head row g0 (and g0 + 4 with two loader warps)
     const int64_t head_stride = static_cast<int64_t>(a.N) * 128;
     int nq = 0;                        // uses of the query ring so far
-    int pend[3] = {0, 0, 0}, np_head = 0, npend = 0;  // filled stages not yet published (FIFO)
+    int pend[kLag + 1] = {}, np_head = 0, npend = 0;  // filled stages not yet published (FIFO)
     int4 inf = info(blockIdx.x);
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
       const Cursor2 c = cursor(item, inf);
@@ -137,16 +138,16 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
           }
         }
         cp_commit();
-        // Publish the stage filled two tiles ago: its copies have landed
-        // (at most two newer groups pending), and the proxy fence makes these
+        // Publish the stage filled kLag tiles ago: its copies have landed
+        // (at most kLag newer groups pending), and the proxy fence makes these
         // generic-proxy writes visible to the tensor cores' async-proxy reads.
-        pend[(np_head + npend) % 3] = qs;
+        pend[(np_head + npend) % (kLag + 1)] = qs;
         ++npend;
-        if (npend > 2) {
-          cp_wait<2>();
+        if (npend > kLag) {
+          cp_wait<kLag>();
           fence_proxy_async();
           mbar_arrive(&qfull[pend[np_head]]);
-          np_head = (np_head + 1) % 3;
+          np_head = (np_head + 1) % (kLag + 1);
           --npend;
         }
         ++nq;
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     fence_proxy_async();
     for (; npend > 0; --npend) {
       mbar_arrive(&qfull[pend[np_head]]);
-      np_head = (np_head + 1) % 3;
+      np_head = (np_head + 1) % (kLag + 1);
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issue
@@ -257,25 +258,26 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       ++na;
       int nv = nkeys;
       if (causal && ok) nv = static_cast<int>(min(static_cast<int64_t>(nv), static_cast<int64_t>(w >> 5) - key0 + 1));
-      float mx = -INFINITY;
+      // Four partial maxima and sums keep the dependent chains short.
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (nv >= 64) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
+        for (int j = 0; j < 64; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
       } else {
 #pragma unroll
         for (int j = 0; j < 64; ++j)
-          if (j < nv) mx = fmaxf(mx, __uint_as_float(v[j]));
+          if (j < nv) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
       }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       const float mxs = mx * sl2;
-      // Four partial sums shorten the dependent add chain.
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
       if (nv >= 64) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) s4[j & 3] += exp2f(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+        for (int j = 0; j < 64; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
       } else {
 #pragma unroll
         for (int j = 0; j < 64; ++j)
-          if (j < nv) s4[j & 3] += exp2f(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+          if (j < nv) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
       }
       const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       float u = ok ? mx * a.scale + logf(sum) : 0.f;

@@ -52,6 +52,15 @@ __device__ inline void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// 2^x by the hardware's approximate base-2 exponential (the PTX ex2.approx
+// instruction, flushing subnormal results to zero): one instruction, relative
+// error near 2^-22, which the LSE epilogues need and nothing more.
+__device__ inline float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (stride byte offset), descriptor version 1.
 __device__ inline uint64_t sw128_desc(uint32_t saddr) {
