@@ -6,20 +6,22 @@
 // One CTA per SM runs a warp-specialised pipeline over the stage-2 work
 // items (64 (query, leaf) pairs of one bucket, walked grid-strided so that
 // all SMs share the current query window in L2):
-//   warps 4-7 (loads): per tile of 16 queries, their 8 head rows
+//   warps 8-11 (loads): per tile of 16 queries, their 8 head rows
 //     (16 x 8 = 128 rows) gathered with 16-byte cp.async straight into the
 //     swizzled operand layout of a ring of query stages, running ahead of the
 //     MMAs (many small bulk copies cost more than one per 2 KB row group);
-//   warp 8, one lane (MMA): per item, the leaf's 64 x 128 key tile by bulk
+//   warp 12, one lane (MMA): per item, the leaf's 64 x 128 key tile by bulk
 //     tensor copy, issued one item ahead into a double buffer; per tile, eight
 //     tcgen05.mma (M = 128 query-head
 //     rows, N = 64 keys, K = 16 each) into a ring of TMEM accumulators,
 //     then tcgen05.commit to release the query stage (and, after an item's
 //     last tile, the key tile) and to publish the accumulator;
-//   warps 0-3 (epilogue): each thread owns one TMEM lane = one (query, head)
-//     row, loads its 64 key scores with tcgen05.ld, takes the LSE over the
-//     usable keys in registers, sums the 8 heads of its query with three
-//     shuffles, and one lane per query stores the leaf score.
+//   warps 0-7 (epilogue): warps w and w + 4 share TMEM lane quarter w; each
+//     thread owns one lane = one (query, head) row and loads 32 of its 64 key
+//     scores with tcgen05.ld; each half takes a partial max and exp-sum over
+//     its usable keys, the halves are combined through shared memory into the
+//     row's LSE, the 8 heads of a query are summed with three shuffles, and
+//     one lane per query stores the leaf score.
 // Operands sit in shared memory as 128-byte-swizzled K-major tiles (rows of
 // 64 bf16, 8-row groups 1 KB apart), which is both the bulk-copy layout and
 // the MMA descriptor layout. Every mbarrier wait is bounded in time; the
@@ -33,8 +35,9 @@ namespace pisa {
 
 namespace {
 
-constexpr int kLoadWarps = 4;              // warps 4-7 gather the query rows
-constexpr int kMmaWarp = 4 + kLoadWarps;   // warp 8 issues the MMAs
+constexpr int kEpiWarps = 8;               // warps 0-7: two per TMEM lane quarter, 32 columns each
+constexpr int kLoadWarps = 4;              // warps 8-11 gather the query rows
+constexpr int kMmaWarp = kEpiWarps + kLoadWarps;  // warp 12 issues the MMAs
 constexpr int kUmmaThreads = 32 * (kMmaWarp + 1);
 constexpr int kLoaders = 32 * kLoadWarps;
 constexpr int kTilePairs = 16;             // queries per MMA tile (x 8 heads = 128 rows)
@@ -56,6 +59,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ uint64_t kfull[2], kempty[2], qfull[kQStages], qempty[kQStages], accfull[kAccStages], accempty[kAccStages];
   __shared__ uint32_t tmem_base_sh;
+  __shared__ float2 xch[2][4][32];  // per tile parity and lane quarter: the second half's (max, sum) per row
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* kbuf = smem;                       // [2][kKeyBytes]
@@ -68,7 +72,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     }
     for (int i = 0; i < kAccStages; ++i) {
       mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], 4);
+      mbar_init(&accempty[i], kEpiWarps);
     }
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&qfull[i], kLoaders);
@@ -100,9 +104,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     return c;
   };
 
-  if (warp >= 4 && warp < kMmaWarp) {
+  if (warp >= kEpiWarps && warp < kMmaWarp) {
     // ---------------------------------------------------------- loads
-    const int lw = warp - 4;                      // loader warp 0..kLoadWarps-1
+    const int lw = warp - kEpiWarps;              // loader warp 0..kLoadWarps-1
     const int jcol = lane & 15;                   // 16-byte column of a 256-byte query row
     const int g0 = 2 * lw + (lane >> 4);          // head row g0 (and g0 + 4 with two loader warps)
     const int64_t head_stride = static_cast<int64_t>(a.N) * 128;
@@ -210,7 +214,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     // Tiles are walked as one stream; each row's (query, slot) word is
     // loaded one tile ahead so its latency hides behind the current tile.
     const float sl2 = a.scale * 1.4426950408889634f;
-    const int row = 32 * warp + lane;  // TMEM lane = (query, head) row of the tile
+    const int qtr = warp & 3, hf = warp >> 2;  // TMEM lane quarter; half of the 64 key columns
+    const int row = 32 * qtr + lane;            // TMEM lane = (query, head) row of the tile
     int na = 0;
     int item = blockIdx.x;
     Cursor2 c = cursor(item, info(item));
@@ -241,16 +246,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       w_next = itemn < total ? pair_word(cn, tln) : 0xffffffffu;
 
       const int as = na % kAccStages;
+      const int xb = na & 1;
       mbar_wait(&accfull[as], (na / kAccStages) & 1, faults);
+      __syncwarp();  // the TMEM load below is warp-collective
       tc_fence_after();
-      uint32_t v[64];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + as * kAccCols;
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-        tmem_ld32(taddr, lo);
-        tmem_ld32(taddr + 32, hi);
-      }
+      uint32_t v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + as * kAccCols + 32 * hf, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -258,35 +259,46 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       ++na;
       int nv = nkeys;
       if (causal && ok) nv = static_cast<int>(min(static_cast<int64_t>(nv), static_cast<int64_t>(w >> 5) - key0 + 1));
-      // Four partial maxima and sums keep the dependent chains short.
+      // This warp's columns [32 hf, 32 hf + 32): partial max and sum of exp
+      // (four chains each), then the two halves of a row are combined.
+      const int nvh = nv - 32 * hf;
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (nv >= 64) {
+      if (nvh >= 32) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
+        for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
       } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
-          if (j < nv) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
+        for (int j = 0; j < 32; ++j)
+          if (j < nvh) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
       }
       const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       const float mxs = mx * sl2;
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (nv >= 64) {
+      if (nvh >= 32) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+        for (int j = 0; j < 32; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
       } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
-          if (j < nv) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+        for (int j = 0; j < 32; ++j)
+          if (j < nvh) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
       }
       const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      float u = ok ? mx * a.scale + logf(sum) : 0.f;
-      u += __shfl_xor_sync(kFull, u, 1);
-      u += __shfl_xor_sync(kFull, u, 2);
-      u += __shfl_xor_sync(kFull, u, 4);
-      if (ok && (row & 7) == 0) {
-        const int64_t orow = bh * a.N + static_cast<int64_t>(w >> 5);
-        ws.score[orow * 32 + (w & 31)] = u;
+      if (hf == 1) xch[xb][qtr][lane] = make_float2(mx, sum);
+      named_sync(1 + qtr, 64);  // the two warps of this lane quarter
+      if (hf == 0) {
+        const float2 o = xch[xb][qtr][lane];
+        const float m = fmaxf(mx, o.x);
+        float z = 0.f;
+        if (mx != -INFINITY) z += sum * ex2_approx((mx - m) * sl2);
+        if (o.x != -INFINITY) z += o.y * ex2_approx((o.x - m) * sl2);
+        float u = ok ? m * a.scale + logf(z) : 0.f;
+        u += __shfl_xor_sync(kFull, u, 1);
+        u += __shfl_xor_sync(kFull, u, 2);
+        u += __shfl_xor_sync(kFull, u, 4);
+        if (ok && (row & 7) == 0) {
+          const int64_t orow = bh * a.N + static_cast<int64_t>(w >> 5);
+          ws.score[orow * 32 + (w & 31)] = u;
+        }
       }
       c = cn;
       tl = tln;

@@ -61,6 +61,11 @@ __device__ inline float ex2_approx(float x) {
   return y;
 }
 
+// Barrier `id` (1..15) among `nthreads` threads of the CTA (whole warps).
+__device__ inline void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (stride byte offset), descriptor version 1.
 __device__ inline uint64_t sw128_desc(uint32_t saddr) {
