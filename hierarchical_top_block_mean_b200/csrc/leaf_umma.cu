@@ -35,7 +35,9 @@ namespace pisa {
 
 namespace {
 
-constexpr int kEpiWarps = 8;               // warps 0-7: two per TMEM lane quarter, 32 columns each
+constexpr int kEpiSplit = 2;               // epilogue warps per TMEM lane quarter (split of the 64 columns)
+constexpr int kEpiWarps = 4 * kEpiSplit;   // warps 0 .. kEpiWarps - 1
+constexpr int kEpiCols = 64 / kEpiSplit;   // key columns per epilogue warp
 constexpr int kLoadWarps = 4;              // warps 8-11 gather the query rows
 constexpr int kMmaWarp = kEpiWarps + kLoadWarps;  // warp 12 issues the MMAs
 constexpr int kUmmaThreads = 32 * (kMmaWarp + 1);
@@ -59,7 +61,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ uint64_t kfull[2], kempty[2], qfull[kQStages], qempty[kQStages], accfull[kAccStages], accempty[kAccStages];
   __shared__ uint32_t tmem_base_sh;
-  __shared__ float2 xch[2][4][32];  // per tile parity and lane quarter: the second half's (max, sum) per row
+  __shared__ float2 xch[2][kEpiSplit - 1][4][32];  // per tile parity, part >= 1 and quarter: (max, sum) per row
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* kbuf = smem;                       // [2][kKeyBytes]
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     // Tiles are walked as one stream; each row's (query, slot) word is
     // loaded one tile ahead so its latency hides behind the current tile.
     const float sl2 = a.scale * 1.4426950408889634f;
-    const int qtr = warp & 3, hf = warp >> 2;  // TMEM lane quarter; half of the 64 key columns
+    const int qtr = warp & 3, hf = warp >> 2;  // TMEM lane quarter; part of the 64 key columns
     const int row = 32 * qtr + lane;            // TMEM lane = (query, head) row of the tile
     int na = 0;
     int item = blockIdx.x;
@@ -250,8 +252,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       mbar_wait(&accfull[as], (na / kAccStages) & 1, faults);
       __syncwarp();  // the TMEM load below is warp-collective
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + as * kAccCols + 32 * hf, v);
+      uint32_t v[kEpiCols];
+      tmem_ld_cols<kEpiCols>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + as * kAccCols + kEpiCols * hf, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -259,38 +261,44 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       ++na;
       int nv = nkeys;
       if (causal && ok) nv = static_cast<int>(min(static_cast<int64_t>(nv), static_cast<int64_t>(w >> 5) - key0 + 1));
-      // This warp's columns [32 hf, 32 hf + 32): partial max and sum of exp
-      // (four chains each), then the two halves of a row are combined.
-      const int nvh = nv - 32 * hf;
+      // This warp's columns [kEpiCols hf, kEpiCols (hf + 1)): partial max and
+      // sum of exp (four chains each), then the parts of a row are combined.
+      const int nvh = nv - kEpiCols * hf;
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (nvh >= 32) {
+      if (nvh >= kEpiCols) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
+        for (int j = 0; j < kEpiCols; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < kEpiCols; ++j)
           if (j < nvh) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
       }
       const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       const float mxs = mx * sl2;
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (nvh >= 32) {
+      if (nvh >= kEpiCols) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+        for (int j = 0; j < kEpiCols; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < kEpiCols; ++j)
           if (j < nvh) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
       }
       const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      if (hf == 1) xch[xb][qtr][lane] = make_float2(mx, sum);
-      named_sync(1 + qtr, 64);  // the two warps of this lane quarter
+      if (hf > 0) xch[xb][hf - 1][qtr][lane] = make_float2(mx, sum);
+      named_sync(1 + qtr, 32 * kEpiSplit);  // the epilogue warps of this lane quarter
       if (hf == 0) {
-        const float2 o = xch[xb][qtr][lane];
-        const float m = fmaxf(mx, o.x);
+        float2 part[kEpiSplit];
+        part[0] = make_float2(mx, sum);
+#pragma unroll
+        for (int i = 1; i < kEpiSplit; ++i) part[i] = xch[xb][i - 1][qtr][lane];
+        float m = part[0].x;
+#pragma unroll
+        for (int i = 1; i < kEpiSplit; ++i) m = fmaxf(m, part[i].x);
         float z = 0.f;
-        if (mx != -INFINITY) z += sum * ex2_approx((mx - m) * sl2);
-        if (o.x != -INFINITY) z += o.y * ex2_approx((o.x - m) * sl2);
+#pragma unroll
+        for (int i = 0; i < kEpiSplit; ++i)
+          if (part[i].x != -INFINITY) z += part[i].y * ex2_approx((part[i].x - m) * sl2);
         float u = ok ? m * a.scale + logf(z) : 0.f;
         u += __shfl_xor_sync(kFull, u, 1);
         u += __shfl_xor_sync(kFull, u, 2);
