@@ -7,15 +7,17 @@
 // queries of one kv head, i.e. 128 (query, head) rows, which stay in shared
 // memory as the MMA's A operand for the CTA's whole life. The leaves stream
 // past it:
-//   warp 4, one lane (loads): each leaf's 64 x 128 key tile by bulk tensor
+//   warp 8, one lane (loads): each leaf's 64 x 128 key tile by bulk tensor
 //     copy into a ring of kKStages buffers;
-//   warp 5, one lane (MMA): per leaf, eight tcgen05.mma (M = 128 rows,
+//   warp 9, one lane (MMA): per leaf, eight tcgen05.mma (M = 128 rows,
 //     N = 64 keys, K = 16) into a ring of TMEM accumulators, then commits that
 //     free the key buffer and publish the accumulator;
-//   warps 0-3 (epilogue): each thread owns one TMEM lane = one (query, head)
-//     row: it loads the 64 logits, takes the LSE over the usable keys, sums
-//     the G_Q heads of its query by shuffles, and the query's first lane keeps
-//     a running top-K list in shared memory (entries are rarely displaced once
+//   warps 0-7 (epilogue): warps w and w + 4 share TMEM lane quarter w; each
+//     thread owns one lane = one (query, head) row and loads 32 of its 64
+//     logits; the two halves' partial max and exp-sum are combined through
+//     shared memory into the row's LSE over the usable keys; the G_Q heads of
+//     a query are summed by shuffles, and the query's first lane keeps a
+//     running top-K list in shared memory (entries are rarely displaced once
 //     the list is full, so the insertion sort costs little).
 // Causal tiles stop at the last leaf their latest query can use and are
 // launched longest first. Every mbarrier wait is bounded in time; the TMEM
@@ -30,7 +32,10 @@ namespace pisa {
 
 namespace {
 
-constexpr int kExThreads = 6 * 32;          // warps 0-3 epilogue, 4 loads, 5 MMA
+constexpr int kExEpiWarps = 8;              // warps 0-7 epilogue (two per TMEM lane quarter)
+constexpr int kExLoadWarp = kExEpiWarps;    // warp 8 loads key tiles
+constexpr int kExMmaWarp = kExEpiWarps + 1; // warp 9 issues the MMAs
+constexpr int kExThreads = 32 * (kExEpiWarps + 2);
 constexpr int kExKStages = 3;               // key tile buffers
 constexpr int kExAccStages = 4;             // TMEM accumulators of 64 columns
 constexpr uint32_t kExTmemCols = kExAccStages * 64;
@@ -52,6 +57,7 @@ __global__ void __launch_bounds__(kExThreads, 2)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ uint64_t kfull[kExKStages], kempty[kExKStages], accfull[kExAccStages], accempty[kExAccStages];
   __shared__ uint32_t tmem_base_sh;
+  __shared__ float2 xch[2][4][32];  // per leaf parity and lane quarter: the second half's (max, sum) per row
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* qbuf = smem;               // A operand, resident
@@ -77,7 +83,7 @@ __global__ void __launch_bounds__(kExThreads, 2)
     }
     for (int i = 0; i < kExAccStages; ++i) {
       mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], 4);
+      mbar_init(&accempty[i], kExEpiWarps);
     }
     mbar_init_fence();
   }
@@ -107,7 +113,7 @@ __global__ void __launch_bounds__(kExThreads, 2)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == 4) {
+  if (warp == kExLoadWarp) {
     // ---------------------------------------------------------- key loads
     if (lane == 0) {
       for (int i = 0; i < nleaf; ++i) {
@@ -119,7 +125,7 @@ __global__ void __launch_bounds__(kExThreads, 2)
         tma_load_2d(kbuf + s * kExKeyBytes + 64 * 128, &tmk, 64, y, &kfull[s]);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kExMmaWarp) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
       const uint32_t qa = smem_u32(qbuf);
@@ -141,11 +147,12 @@ __global__ void __launch_bounds__(kExThreads, 2)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    const int row = 32 * warp + lane;
+    const int qtr = warp & 3, hf = warp >> 2;  // TMEM lane quarter; half of the 64 key columns
+    const int row = 32 * qtr + lane;
     const int qi = row / G;
     const int64_t t = t0 + qi;
     const bool qok = t < N;
-    const bool owner = (row % G) == 0;
+    const bool owner = hf == 0 && (row % G) == 0;
     const int K = a.K;
     const float sl2 = a.scale * 1.4426950408889634f;
     float* rs = ls + qi * kMaxK;
@@ -157,14 +164,8 @@ __global__ void __launch_bounds__(kExThreads, 2)
       mbar_wait(&accfull[as], (i / kExAccStages) & 1, faults);
       __syncwarp();  // the TMEM load below is warp-collective
       tc_fence_after();
-      uint32_t v[64];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + as * 64;
-      {
-        uint32_t(&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-        uint32_t(&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-        tmem_ld32(taddr, lo);
-        tmem_ld32(taddr + 32, hi);
-      }
+      uint32_t v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + as * 64 + 32 * hf, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -174,29 +175,42 @@ __global__ void __launch_bounds__(kExThreads, 2)
       int64_t lim = N - key0;
       if (causal && t - key0 + 1 < lim) lim = t - key0 + 1;
       const int nv = qok ? static_cast<int>(lim < 0 ? 0 : (lim > 64 ? 64 : lim)) : 0;
+      // This warp's half of the columns: partial max and exp-sum, then the
+      // halves of a row are combined through shared memory.
+      const int nvh = nv - 32 * hf;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (nvh >= 32) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvh) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
+      }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      const float mxs = mx * sl2;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (nvh >= 32) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvh) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+      }
+      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      const int xb = i & 1;
+      if (hf == 1) xch[xb][qtr][lane] = make_float2(mx, sum);
+      named_sync(1 + qtr, 64);  // the two warps of this lane quarter
+      if (hf == 1) continue;
       float u = 0.f;
       if (nv > 0) {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (nv >= 64) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (j < nv) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
-        }
-        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        const float mxs = mx * sl2;
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (nv >= 64) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (j < nv) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
-        }
-        u = mx * a.scale + logf((s4[0] + s4[1]) + (s4[2] + s4[3]));
+        const float2 o = xch[xb][qtr][lane];
+        const float m = fmaxf(mx, o.x);
+        float z = 0.f;
+        if (mx != -INFINITY) z += sum * ex2_approx((mx - m) * sl2);
+        if (o.x != -INFINITY) z += o.y * ex2_approx((o.x - m) * sl2);
+        u = m * a.scale + logf(z);
       }
       // The G rows of a query are G consecutive lanes and share nv.
 #pragma unroll
