@@ -38,6 +38,10 @@ pisa_status check_cfg(const pisa_config* c) {
   pisa_status s = check_shape(c->H_q, c->H_kv, c->d, c->C, c->g, c->K, c->dtype);
   if (s != PISA_OK) return s;
   if (c->q_tile != 4) return PISA_ERR_UNSUPPORTED;
+  // Tensor-map row coordinates are 32-bit, and a stage-2 pair packs its query
+  // position into 27 bits.
+  if (static_cast<int64_t>(c->B) * c->H_q * c->N >= (int64_t{1} << 31) || c->N >= (1 << 27))
+    return PISA_ERR_UNSUPPORTED;
   return PISA_OK;
 }
 

@@ -31,7 +31,8 @@
  *     returns PISA_ERR_CUDA. Nothing in the library traps or waits without a
  *     bound.
  *   - Supported shapes: g = 2; C in {32, 64}; d in {64, 128}; 1 <= K <= 16;
- *     q_tile = 4; G_Q in {1, 2, 4, 8}; other values return
+ *     q_tile = 4; G_Q in {1, 2, 4, 8}; for the prefill calls also
+ *     B * H_q * N < 2^31 and N < 2^27. Other values return
  *     PISA_ERR_UNSUPPORTED.
  */
 #ifndef PISA_H_

@@ -54,6 +54,7 @@ def _cfg(**kw):
 
 
 @pytest.mark.parametrize("kw,code", [
+    (dict(N=1 << 27), 2), (dict(B=64, N=1 << 22, H_q=8), 2),
     (dict(N=0), 1), (dict(B=0), 1), (dict(H_q=6, H_kv=4), 1), (dict(dtype=7), 1), (dict(causal=2), 1),
     (dict(g=3), 2), (dict(C=16), 2), (dict(d=96), 2), (dict(K=17), 2), (dict(q_tile=8), 2),
     (dict(H_q=12, H_kv=1), 2),
@@ -67,7 +68,11 @@ def test_invalid_configs_rejected_before_launch(kw, code):
     assert lib.pisa_select(ctypes.byref(cfg), dummy, dummy, dummy, dummy, None, dummy, 1 << 30, None) == code
     assert lib.pisa_select_flat(ctypes.byref(cfg), dummy, dummy, dummy, None) == code
     assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), dummy, dummy, dummy, dummy, dummy, None, None) == code
+    assert lib.pisa_select_exact(ctypes.byref(cfg), dummy, dummy, dummy, None) == code
+    assert lib.pisa_sparse_attn_bwd(ctypes.byref(cfg), dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy,
+                                    dummy, dummy, 1 << 30, None) == code
     assert lib.pisa_select_workspace_bytes(ctypes.byref(cfg)) == 0
+    assert lib.pisa_attn_bwd_workspace_bytes(ctypes.byref(cfg)) == 0
     assert lib.pisa_launch_count() == before
 
 
