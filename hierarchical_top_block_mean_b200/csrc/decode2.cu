@@ -16,8 +16,9 @@
 //   stream through a per-warp ring of shared-memory tiles (16 keys x d each,
 //   filled by cp.async ahead of use, so every warp keeps loads in flight) and
 //   S^T = K Q^T is taken per tile on tensor cores. The scaled logits of every
-//   candidate key are kept in shared memory. Top-K by warp bitonic sort; ties
-//   to the lower block index.
+//   candidate key go to the caller's workspace (a few tens of KB per CTA,
+//   read back from L2). Top-K by warp bitonic sort; ties to the lower block
+//   index.
 // * Attend. The logits of the selected blocks are among those just computed
 //   for the leaf level, so only V streams through the ring: O^T += V^T P^T
 //   per 16-key tile under an online softmax, and the warps' partial states
@@ -27,6 +28,9 @@
 // * Lengths. With append, the H_kv CTAs of a sequence form one thread-block
 //   cluster: all of them read len[s] before the cluster barrier, after which
 //   the first CTA stores len[s] + 1.
+// * Caches. Dense [S, H_kv, cap, d], or paged (PAGED): leaf i of sequence s
+//   in page block_table[s][i] of a pool [pages, H_kv, C, d]. Only the row
+//   address differs (kv_row); the arithmetic and its order are the same.
 #include <cooperative_groups.h>
 
 #include "attn_mma.cuh"
