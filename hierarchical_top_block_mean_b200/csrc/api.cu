@@ -1,6 +1,6 @@
 // C ABI entry points (include/pisa.h): host-side validation, layout
 // arithmetic and dispatch to the kernels. Nothing here allocates device
-// memory, synchronises or keeps state besides the launch counter.
+// memory or synchronises; the only state is the launch counter.
 #include <atomic>
 #include <cmath>
 

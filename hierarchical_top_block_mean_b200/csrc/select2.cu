@@ -3,11 +3,14 @@
 //   stage 1  router_kernel     one warp per (kv head, query): levels L..2 of
 //                              the coarse-to-fine search; candidate children
 //                              scored on tensor cores.
-//   grouping count (in stage 1), scan_kernel, scatter_kernel: a CSR of the
-//                              (query, candidate leaf) pairs keyed by leaf.
-//   stage 2  leaf_kernel       per leaf bucket: the C x d key tile is staged
-//                              in shared memory once and reused across tiles
-//                              of Q_tile = 4 queries x G_Q heads
+//   grouping count (in stage 1), scan_kernel, scatter_kernel,
+//                              itemize_kernel: a CSR of the (query, candidate
+//                              leaf) pairs keyed by (kv head, query window,
+//                              leaf), cut into work items of 64 pairs.
+//   stage 2  leaf_umma_kernel  (leaf_umma.cu; G_Q = 8, d = 128, C = 64) or
+//            leaf_kernel       per work item: the C x d key tile is brought
+//                              into shared memory once and reused across
+//                              tiles of the item's queries x G_Q heads
 //                              ((Q_tile G_Q) x d . d x C on tensor cores),
 //                              then a per-head LSE over the keys and a sum
 //                              over the G_Q heads.
