@@ -289,10 +289,25 @@ def time_decode(wd, steps=32, warmup=4):
     e1.record()
     torch.cuda.synchronize()
     us_sel = e0.elapsed_time(e1) * 1e3 / steps
+    # Attention alone over the selection just made, then the append alone
+    # (each its own launch; the append advances every sequence by one token).
+    e0.record()
+    for _ in range(steps):
+        st.attend(q)
+    e1.record()
+    torch.cuda.synchronize()
+    us_attn = e0.elapsed_time(e1) * 1e3 / steps
+    e0.record()
+    for s in range(steps):
+        st.append(ins[s][1], ins[s][2])
+    e1.record()
+    torch.cuda.synchronize()
+    us_app = e0.elapsed_time(e1) * 1e3 / steps
     ok = int(st.status.item()) == 0
     del st, kc, vc
     torch.cuda.empty_cache()
-    return {"workload": wd.name, "us_per_step": us, "select_us": us_sel, "steps": steps, "status_ok": ok}
+    return {"workload": wd.name, "us_per_step": us, "select_us": us_sel, "attn_us": us_attn, "append_us": us_app,
+            "steps": steps, "status_ok": ok}
 
 
 def time_decode_paged(wd, steps=32, warmup=4):
