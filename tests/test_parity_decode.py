@@ -58,6 +58,12 @@ SMALL = [
                                              d=64, C=32, K=5, seed=5200),
     workloads.DECODE["decode_64x128k"].with_(name="dec_small_f32", S=2, context=60, steps=80, H_q=4, H_kv=1, d=64,
                                              C=32, K=4, dtype="f32", seed=5300),
+    workloads.DECODE["decode_64x128k"].with_(name="dec_small_G8", S=2, context=500, steps=40, H_q=16, H_kv=2,
+                                             seed=5400),
+    workloads.DECODE["decode_64x128k"].with_(name="dec_small_G1", S=2, context=420, steps=30, H_q=4, H_kv=4,
+                                             K=8, seed=5500),
+    workloads.DECODE["decode_64x128k"].with_(name="dec_small_G2_d64", S=3, context=200, steps=30, H_q=8, H_kv=4,
+                                             d=64, C=32, K=3, seed=5600),
 ]
 
 

@@ -15,6 +15,8 @@ CASES = [
     workloads.DECODE["decode_64x128k"].with_(name="paged_C64_d128", S=5, context=900, steps=40, seed=7100),
     workloads.DECODE["decode_64x128k"].with_(name="paged_C32_d64_G4", S=4, context=300, steps=50, H_q=8, H_kv=2,
                                              d=64, C=32, K=5, seed=7200),
+    workloads.DECODE["decode_64x128k"].with_(name="paged_G8_K16", S=3, context=700, steps=30, H_q=16, H_kv=2,
+                                             seed=7300),
 ]
 
 
