@@ -7,11 +7,13 @@ heads, 2 kv heads, d = 128, C = 64, K = 16, bf16, causal, 256 planted
 needles). The flat single-level selector and the decode step (64 sequences x
 131072 cached tokens) are timed beside it and reported in the same line.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--seq-parallel]
 
 Under torchrun each rank runs the same workload on its own GPU (weak
 scaling: the path shards over independent sequences and heads with no
-collective); the barrier-bracketed time is the max over ranks.
+collective); the barrier-bracketed time is the max over ranks. With
+--seq-parallel the ranks instead split one sequence by position and
+all-gather its keys and values over NCCL (strong scaling).
 """
 from __future__ import annotations
 
@@ -30,7 +32,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from hierarchical_top_block_mean_b200 import api, workloads  # noqa: E402
+from hierarchical_top_block_mean_b200 import api, seqpar, workloads  # noqa: E402
 
 METRIC = "PISA prefill tokens/s (select+attn) at 64K/256K; decode select µs/step"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -424,6 +426,31 @@ def run_gpu(args):
     if needles:
         needles["flat"] = needle_recall(p.sel, x["needles"])
 
+    # Sequence-parallel split of the step over 8 GPUs, each GPU's share
+    # timed here one after another on this GPU: the pyramid over all keys,
+    # then the selection and attention of its eighth of the query rows. The
+    # key and value all-gather that precedes them is not in these figures.
+    seq_par = None
+    if w.N % 8 == 0:
+        shard_ms = []
+        for r in range(8):
+            a, n = seqpar.shard_span(w.N, 8, r)
+            qs = q[:, :, a:a + n].contiguous()
+            sh = api.PrefillShard(pr, a, n, dev)
+            sh(qs, k, v)
+            se0, se1 = events(2)
+            se0.record(stream)
+            sh(qs, k, v)
+            se1.record(stream)
+            torch.cuda.synchronize()
+            shard_ms.append(se0.elapsed_time(se1))
+            del qs, sh
+        seq_par = {"shards": 8, "shard_ms": shard_ms, "max_shard_ms": max(shard_ms),
+                   "balance": max(shard_ms) / (sum(shard_ms) / len(shard_ms)),
+                   "note": "per-GPU compute of an 8-way sequence-parallel step (pyramid over all keys + "
+                           "selection and attention of 1/8 of the queries), each shard timed once on this "
+                           "GPU after a warm-up; the NVLink all-gather of K and V is not included"}
+
     # Attention backward over the step's selection (training), once after a
     # warm-up: dq, dk, dv (fp32) for a random output gradient.
     bwd_ms = None
@@ -493,6 +520,7 @@ def run_gpu(args):
         "pisa_recall_vs_exact": recall,
         "needle_recall": needles,
         "attn_bwd_ms": bwd_ms,
+        "seq_parallel": seq_par,
         "decode": decode,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -508,6 +536,86 @@ def run_gpu(args):
     return 0
 
 
+def run_seq_parallel(args):
+    """One sequence split by position over the ranks (strong scaling): per
+    step, the NCCL all-gather of the key and value slices, the pyramid, and
+    the selection and attention of each rank's query rows
+    (seqpar.SeqParallelPrefill). Without torchrun it runs one rank."""
+    import datetime
+
+    import torch.distributed as tdist
+    dist = dist_init(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if dist is None:
+        tdist.init_process_group("nccl", store=tdist.HashStore(), rank=0, world_size=1, device_id=dev,
+                                 timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    rank, world = dist.get_rank(), dist.get_world_size()
+    w = workloads.PREFILL[args.workload]
+    x = workloads.prefill_inputs(w, device=dev)  # the same seeded sequence on every rank
+    q0, n = seqpar.shard_span(w.N, world, rank)
+    q, k, v = (x[t][:, :, q0:q0 + n].contiguous() for t in ("q", "k", "v"))
+    pr = api.Problem.of(x["q"], x["k"], C=w.C, K=w.K, causal=w.causal)
+    del x
+    torch.cuda.empty_cache()
+    sp = seqpar.SeqParallelPrefill(pr, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        sp(q, k, v)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = api.launch_count()
+    e0, e1 = events(2)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            sp(q, k, v)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+    launches = api.launch_count() - launches0
+    ms = max_over_ranks(dist, e0.elapsed_time(e1) / args.steps)
+    value = w.B * w.N / (ms * 1e-3)  # the whole sequence's tokens per step
+
+    # End to end: this rank's slices from pinned host memory, its output rows back.
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = torch.empty(sp.shard.out.shape, dtype=sp.shard.out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    e2e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    dist.barrier()
+    ee0, ee1 = events(2)
+    ee0.record(stream)
+    for _ in range(e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        sp(dq, dk, dv)
+        hout.copy_(sp.shard.out, non_blocking=True)
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(dist, ee0.elapsed_time(ee1) / e2e_steps)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = hout.numel() * hout.element_size()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "C": w.C,
+                   "g": 2, "K": w.K, "q_tile": 4, "causal": w.causal, "parallelism": f"sp{world}",
+                   "tokens_per_rank": n, "l2": "inputs larger than L2"},
+        "e2e": {"value": w.B * w.N / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "per": "rank"},
+        "gpu_launches": launches, "roofline": None, "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    del sp
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -517,6 +625,9 @@ def main():
     ap.add_argument("--workload", default="needle_256k", choices=sorted(workloads.PREFILL))
     ap.add_argument("--decode-workload", default="decode_64x128k", choices=sorted(workloads.DECODE))
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--seq-parallel", action="store_true",
+                    help="split one sequence over the ranks by position (strong scaling) instead of a full "
+                         "sequence per rank")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-step-budget", type=float, default=None,
@@ -525,6 +636,8 @@ def main():
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.seq_parallel:
+        return run_seq_parallel(args)
     return run_gpu(args)
 
 

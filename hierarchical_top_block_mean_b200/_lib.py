@@ -32,6 +32,11 @@ class Config(ctypes.Structure):
                                                "dtype")] + [("scale", ctypes.c_float)]
 
 
+class QuerySpan(ctypes.Structure):
+    """Mirror of pisa_query_span."""
+    _fields_ = [("q0", ctypes.c_int32), ("n_q", ctypes.c_int32)]
+
+
 class DecodeConfig(ctypes.Structure):
     """Mirror of pisa_decode_config."""
     _fields_ = [(n, ctypes.c_int32) for n in ("S", "cap", "H_q", "H_kv", "d", "C", "g", "K", "dtype")] + [
@@ -39,6 +44,7 @@ class DecodeConfig(ctypes.Structure):
 
 
 _PC = ctypes.POINTER(Config)
+_PS = ctypes.POINTER(QuerySpan)
 _PD = ctypes.POINTER(DecodeConfig)
 
 SIGNATURES = {
@@ -57,6 +63,9 @@ SIGNATURES = {
     "pisa_sparse_attn_bwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
     "pisa_sparse_attn_fwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p]),
     "pisa_select_noalloc": (_i32, [_PC, _p, _p, _p, _p, _p, _p]),
+    "pisa_select_span_workspace_bytes": (ctypes.c_size_t, [_PC, _PS]),
+    "pisa_select_span": (_i32, [_PC, _PS, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
+    "pisa_sparse_attn_fwd_span": (_i32, [_PC, _PS, _p, _p, _p, _p, _p, _p, _p]),
     "pisa_decode_pyramid_rows": (_i64, [_PD]),
     "pisa_decode_workspace_bytes": (_i64, [_PD]),
     "pisa_decode_init": (_i32, [_PD, _p, _p, _p, _p]),

@@ -187,6 +187,52 @@ def sparse_attn_fwd(q, k, v, sel, *, C: int, causal: bool, scale: float = 0.0, o
     return out, lse
 
 
+def _span_problem(q, k, C, K, causal, scale):
+    B, H_q, n_q, d = q.shape
+    Bk, H_kv, N, dk = k.shape
+    if (B, d) != (Bk, dk) or q.dtype != k.dtype or q.dtype not in _DT:
+        raise ValueError(f"q {tuple(q.shape)} {q.dtype} and k {tuple(k.shape)} {k.dtype} disagree")
+    return Problem(B, N, H_q, H_kv, d, C, K, bool(causal), q.dtype, scale), n_q
+
+
+def select_span(q, k, pyr, *, q0: int, C: int, K: int, causal: bool, scale: float = 0.0, out=None, score=None,
+                workspace=None):
+    """Selection for the query rows at positions [q0, q0 + n_q) of a sequence:
+    q [B, H_q, n_q, d] holds those rows only; k [B, H_kv, N, d] and pyr cover
+    all N tokens. Returns sel [B, H_kv, n_q, K], equal to those rows of a
+    whole-sequence selection."""
+    for t, n in ((q, "q"), (k, "k"), (pyr, "pyr")):
+        _need(t, n)
+    pr, n_q = _span_problem(q, k, C, K, causal, scale)
+    cfg, span = pr.cstruct(), _lib.QuerySpan(q0, n_q)
+    if out is None:
+        out = torch.empty((pr.B, pr.H_kv, n_q, K), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        need = int(_lib.lib().pisa_select_span_workspace_bytes(ctypes.byref(cfg), ctypes.byref(span)))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _lib.call("pisa_select_span", ctypes.byref(cfg), ctypes.byref(span), _p(q), _p(k), _p(pyr), _p(out), _p(score),
+              _p(workspace), workspace.numel() * workspace.element_size(), _stream(q))
+    return out
+
+
+def sparse_attn_fwd_span(q, k, v, sel, *, q0: int, C: int, causal: bool, scale: float = 0.0, out=None, lse=None,
+                         want_lse: bool = True):
+    """Block-sparse attention for the query rows at positions [q0, q0 + n_q):
+    q [B, H_q, n_q, d] and sel [B, H_kv, n_q, K] hold those rows; k and v all
+    N tokens. Returns (out [B, H_q, n_q, d], lse [B, H_q, n_q] or None)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    _need(sel, "sel", torch.int32)
+    pr, n_q = _span_problem(q, k, C, sel.shape[-1], causal, scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    _lib.call("pisa_sparse_attn_fwd_span", ctypes.byref(pr.cstruct()), ctypes.byref(_lib.QuerySpan(q0, n_q)), _p(q),
+              _p(k), _p(v), _p(sel), _p(out), _p(lse), _stream(q))
+    return out, lse
+
+
 class Prefill:
     """Reusable prefill pipeline for one problem shape: pyramid, PISA select
     and block-sparse attention, with all buffers allocated once."""
@@ -211,6 +257,44 @@ class Prefill:
     def attend(self, q, k, v):
         _lib.call("pisa_sparse_attn_fwd", ctypes.byref(self.cfg), _p(q), _p(k), _p(v), _p(self.sel), _p(self.out),
                   _p(self.lse), _stream(q))
+
+    def __call__(self, q, k, v):
+        self.pyramid(k)
+        self.select(q, k)
+        self.attend(q, k, v)
+        return self.out
+
+
+class PrefillShard:
+    """Prefill of the query rows at positions [q0, q0 + n_q) of an N-token
+    sequence (pr describes the whole sequence): the pyramid over all N keys,
+    then the selection and attention of this shard's rows only, with buffers
+    allocated once. q is [B, H_q, n_q, d]; k and v are [B, H_kv, N, d]."""
+
+    def __init__(self, pr: Problem, q0: int, n_q: int, device="cuda"):
+        self.pr, self.q0, self.n_q = pr, q0, n_q
+        dev = torch.device(device)
+        self.cfg = pr.cstruct()
+        self.span = _lib.QuerySpan(q0, n_q)
+        nbytes = int(_lib.lib().pisa_select_span_workspace_bytes(ctypes.byref(self.cfg), ctypes.byref(self.span)))
+        if pr.dtype == torch.bfloat16 and nbytes == 0:
+            raise ValueError(f"query span [{q0}, {q0 + n_q}) does not fit N = {pr.N}")
+        self.pyr = torch.empty((pr.B, pr.H_kv, pr.R, pr.d), dtype=torch.float32, device=dev)
+        self.sel = torch.empty((pr.B, pr.H_kv, n_q, pr.K), dtype=torch.int32, device=dev)
+        self.ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        self.out = torch.empty((pr.B, pr.H_q, n_q, pr.d), dtype=pr.dtype, device=dev)
+        self.lse = torch.empty((pr.B, pr.H_q, n_q), dtype=torch.float32, device=dev)
+
+    def pyramid(self, k):
+        _lib.call("pisa_build_pyramid", ctypes.byref(self.cfg), _p(k), _p(self.pyr), _stream(k))
+
+    def select(self, q, k):
+        _lib.call("pisa_select_span", ctypes.byref(self.cfg), ctypes.byref(self.span), _p(q), _p(k), _p(self.pyr),
+                  _p(self.sel), None, _p(self.ws), self.ws.numel(), _stream(q))
+
+    def attend(self, q, k, v):
+        _lib.call("pisa_sparse_attn_fwd_span", ctypes.byref(self.cfg), ctypes.byref(self.span), _p(q), _p(k), _p(v),
+                  _p(self.sel), _p(self.out), _p(self.lse), _stream(q))
 
     def __call__(self, q, k, v):
         self.pyramid(k)

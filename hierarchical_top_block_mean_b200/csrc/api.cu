@@ -52,9 +52,17 @@ pisa_status check_dcfg(const pisa_decode_config* c) {
 }
 
 PrefillArgs args_of(const pisa_config* c) {
-  PrefillArgs a{c->B, c->N, c->H_q, c->H_kv, c->d, c->C, c->K, c->causal, c->dtype, c->scale};
+  PrefillArgs a{c->B, c->N, c->H_q, c->H_kv, c->d, c->C, c->K, c->causal, c->dtype, c->scale, 0, c->N};
   if (!(a.scale > 0.f)) a.scale = 1.0f / std::sqrt(static_cast<float>(c->d));
   return a;
+}
+
+// Query span check; narrows a to the span's rows.
+pisa_status apply_span(const pisa_query_span* sp, int N, PrefillArgs* a) {
+  if (!sp || sp->q0 < 0 || sp->n_q < 1 || static_cast<int64_t>(sp->q0) + sp->n_q > N) return PISA_ERR_INVALID_ARGUMENT;
+  a->q0 = sp->q0;
+  a->Nq = sp->n_q;
+  return PISA_OK;
 }
 
 DecodeArgs dargs_of(const pisa_decode_config* c) {
@@ -127,19 +135,29 @@ pisa_status pisa_build_pyramid(const pisa_config* cfg, const void* k, float* pyr
                                         cfg->B * cfg->H_kv, cfg->H_kv, cfg->N, cfg->C, as_stream(stream)));
 }
 
-size_t pisa_select_workspace_bytes(const pisa_config* cfg) {
+size_t pisa_select_span_workspace_bytes(const pisa_config* cfg, const pisa_query_span* span) {
   if (check_cfg(cfg) != PISA_OK) return 0;
   if (cfg->dtype != PISA_DTYPE_BF16) return 0;  // the fp32 path selects row by row without scratch
-  return select2_workspace_bytes(args_of(cfg));
+  PrefillArgs a = args_of(cfg);
+  if (apply_span(span, cfg->N, &a) != PISA_OK) return 0;
+  return select2_workspace_bytes(a);
 }
 
-pisa_status pisa_select(const pisa_config* cfg, const void* q, const void* k, const float* pyr, int32_t* sel,
-                        float* sel_score, void* ws, size_t ws_bytes, void* stream) {
+size_t pisa_select_workspace_bytes(const pisa_config* cfg) {
+  if (check_cfg(cfg) != PISA_OK) return 0;
+  const pisa_query_span all{0, cfg->N};
+  return pisa_select_span_workspace_bytes(cfg, &all);
+}
+
+pisa_status pisa_select_span(const pisa_config* cfg, const pisa_query_span* span, const void* q, const void* k,
+                             const float* pyr, int32_t* sel, float* sel_score, void* ws, size_t ws_bytes,
+                             void* stream) {
   pisa_status s = check_cfg(cfg);
   if (s != PISA_OK) return s;
   if (!q || !k || !pyr || !sel || !aligned16(q) || !aligned16(k) || !aligned16(pyr) || !aligned16(sel))
     return PISA_ERR_INVALID_ARGUMENT;
-  const PrefillArgs a = args_of(cfg);
+  PrefillArgs a = args_of(cfg);
+  if ((s = apply_span(span, cfg->N, &a)) != PISA_OK) return s;
   const Layout lay = make_layout(cfg->N, cfg->C);
   if (cfg->dtype == PISA_DTYPE_BF16) {
     const size_t need = select2_workspace_bytes(a);
@@ -147,6 +165,14 @@ pisa_status pisa_select(const pisa_config* cfg, const void* q, const void* k, co
     return from_cuda(launch_select2(a, q, k, pyr, lay, sel, sel_score, ws, as_stream(stream)));
   }
   return from_cuda(launch_select_rows(a, q, k, pyr, lay, sel, sel_score, as_stream(stream)));
+}
+
+pisa_status pisa_select(const pisa_config* cfg, const void* q, const void* k, const float* pyr, int32_t* sel,
+                        float* sel_score, void* ws, size_t ws_bytes, void* stream) {
+  pisa_status s = check_cfg(cfg);
+  if (s != PISA_OK) return s;
+  const pisa_query_span all{0, cfg->N};
+  return pisa_select_span(cfg, &all, q, k, pyr, sel, sel_score, ws, ws_bytes, stream);
 }
 
 pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float* pyr, int32_t* sel, void* stream) {
@@ -167,15 +193,25 @@ pisa_status pisa_select_exact(const pisa_config* cfg, const void* q, const void*
   return from_cuda(launch_exact_rows(a, q, k, sel, as_stream(stream)));
 }
 
-pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
-                                 const int32_t* sel, void* out, float* lse, void* stream) {
+pisa_status pisa_sparse_attn_fwd_span(const pisa_config* cfg, const pisa_query_span* span, const void* q,
+                                      const void* k, const void* v, const int32_t* sel, void* out, float* lse,
+                                      void* stream) {
   pisa_status s = check_cfg(cfg);
   if (s != PISA_OK) return s;
   if (!q || !k || !v || !sel || !out) return PISA_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return PISA_ERR_INVALID_ARGUMENT;
-  if (cfg->dtype == PISA_DTYPE_BF16)
-    return from_cuda(launch_attn_mma(args_of(cfg), q, k, v, sel, out, lse, as_stream(stream)));
-  return from_cuda(launch_attn_rows(args_of(cfg), q, k, v, sel, out, lse, as_stream(stream)));
+  PrefillArgs a = args_of(cfg);
+  if ((s = apply_span(span, cfg->N, &a)) != PISA_OK) return s;
+  if (cfg->dtype == PISA_DTYPE_BF16) return from_cuda(launch_attn_mma(a, q, k, v, sel, out, lse, as_stream(stream)));
+  return from_cuda(launch_attn_rows(a, q, k, v, sel, out, lse, as_stream(stream)));
+}
+
+pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
+                                 const int32_t* sel, void* out, float* lse, void* stream) {
+  pisa_status s = check_cfg(cfg);
+  if (s != PISA_OK) return s;
+  const pisa_query_span all{0, cfg->N};
+  return pisa_sparse_attn_fwd_span(cfg, &all, q, k, v, sel, out, lse, stream);
 }
 
 size_t pisa_attn_bwd_workspace_bytes(const pisa_config* cfg) {

@@ -35,7 +35,7 @@ constexpr float kLazy = 8.f;  // headroom of the lazily moved softmax maximum (n
 // per lane, held in a register), position in that list and chunk.
 struct Cursor {
   int64_t row;  // -1: exhausted
-  int bh, t;    // row = bh * N + t (divided once per row)
+  int bh, t;    // row = bh * Nq + t: t is the query's row, q0 + t its position (divided once per row)
   int blk_lane; // this lane's entry of the row's compacted block list
   int nblk;     // blocks in the list
   int idx;      // position in the list
@@ -64,8 +64,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   }
   __syncwarp();
   uint32_t phase = 0;  // parity bit of each stage's next completion
-  const int64_t n = a.N;
-  const int64_t rows = static_cast<int64_t>(a.B) * a.H_kv * n;
+  const int64_t n = a.N, nq = a.Nq;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.H_kv * nq;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kAttnWarps;
   const bool causal = a.causal != 0;
 
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
           }
         }
       }
-      return Cursor{r, static_cast<int>(r / n), static_cast<int>(r % n), out_b, __popc(m), 0, 0};
+      return Cursor{r, static_cast<int>(r / nq), static_cast<int>(r % nq), out_b, __popc(m), 0, 0};
     }
     return Cursor{-1, 0, 0, -1, 0, 0, 0};
   };
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       hb = cur.bh / a.H_kv;
       hh = cur.bh % a.H_kv;
       row_now = cur.row;
-      const bf16* qp = q + ((static_cast<int64_t>(hb) * a.H_q + hh * G + (gid < G ? gid : 0)) * n + t) * D + 2 * tig;
+      const bf16* qp = q + ((static_cast<int64_t>(hb) * a.H_q + hh * G + (gid < G ? gid : 0)) * nq + t) * D + 2 * tig;
 #pragma unroll
       for (int ks = 0; ks < kKS; ++ks) {
         qb[ks][0] = gid < G ? *reinterpret_cast<const uint32_t*>(qp + 16 * ks) : 0u;
@@ -155,7 +155,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 #pragma unroll
       for (int i = 0; i < kKS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     }
-    const int last = (causal && cur.t < n - 1) ? cur.t : static_cast<int>(n - 1);  // positions fit int32
+    const int pos = a.q0 + cur.t;  // the query's position; positions fit int32
+    const int last = (causal && pos < n - 1) ? pos : static_cast<int>(n - 1);
     const int blk = __shfl_sync(kFull, cur.blk_lane, cur.idx);
     const int key0 = blk * CC + cur.half * kKeysPerChunk;
     const bool full = key0 + kKeysPerChunk - 1 <= last;
@@ -252,8 +253,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         l[j] += __shfl_xor_sync(kFull, l[j], 8);
         l[j] += __shfl_xor_sync(kFull, l[j], 16);
       }
-      const int64_t hs = n * D;
-      bf16* o0 = out + ((static_cast<int64_t>(hb) * a.H_q + hh * G) * n + t) * D;
+      const int64_t hs = nq * D;
+      bf16* o0 = out + ((static_cast<int64_t>(hb) * a.H_q + hh * G) * nq + t) * D;
       float inv[2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) inv[j] = l[j] > 0.f ? 1.f / l[j] : 0.f;
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       if (lse && gid == 0) {
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-          if (2 * tig + j < G) lse[(static_cast<int64_t>(hb) * a.H_q + hh * G + 2 * tig + j) * n + t] = m[j] + logf(l[j]);
+          if (2 * tig + j < G) lse[(static_cast<int64_t>(hb) * a.H_q + hh * G + 2 * tig + j) * nq + t] = m[j] + logf(l[j]);
       }
     }
     cur = nxt;
@@ -292,12 +293,13 @@ int sm_count_attn() {
 
 cudaError_t launch_attn_mma(const PrefillArgs& a, const void* q, const void* k, const void* v, const int32_t* sel,
                             void* out, float* lse, cudaStream_t st) {
-  const int64_t rows = static_cast<int64_t>(a.B) * a.H_kv * a.N;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.H_kv * a.Nq;      // query rows
+  const int64_t key_rows = static_cast<int64_t>(a.B) * a.H_kv * a.N;   // K and V rows
   const int64_t want = (rows + kAttnWarps - 1) / kAttnWarps;
   const unsigned grid = static_cast<unsigned>(want < sm_count_attn() ? want : sm_count_attn());
   CUtensorMap tmk, tmv;
-  cudaError_t e = make_tmap_bf16_2d(&tmk, k, a.d, static_cast<uint64_t>(rows), kKeysPerChunk);
-  if (e == cudaSuccess) e = make_tmap_bf16_2d(&tmv, v, a.d, static_cast<uint64_t>(rows), kKeysPerChunk);
+  cudaError_t e = make_tmap_bf16_2d(&tmk, k, a.d, static_cast<uint64_t>(key_rows), kKeysPerChunk);
+  if (e == cudaSuccess) e = make_tmap_bf16_2d(&tmv, v, a.d, static_cast<uint64_t>(key_rows), kKeysPerChunk);
   if (e != cudaSuccess) return e;
   unsigned long long* faults = wait_fault_counter();
   return dispatch_tdg(PISA_DTYPE_BF16, a.d, a.H_q / a.H_kv, [&](auto, auto dd, auto gg) -> cudaError_t {

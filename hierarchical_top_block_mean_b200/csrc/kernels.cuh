@@ -10,6 +10,11 @@ namespace pisa {
 struct PrefillArgs {
   int B, N, H_q, H_kv, d, C, K, causal, dtype;
   float scale;
+  // Query rows of the q, sel, out and lse arrays: positions [q0, q0 + Nq)
+  // of the N-key sequence (a whole sequence: q0 = 0, Nq = N). The
+  // selection and forward attention kernels honour them; the flat, exact and
+  // backward kernels take whole sequences only.
+  int q0, Nq;
 };
 
 // Decode problem with the scale resolved.

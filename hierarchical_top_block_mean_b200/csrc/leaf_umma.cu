@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const int lw = warp - kEpiWarps;              // loader warp 0..kLoadWarps-1
     const int jcol = lane & 15;                   // 16-byte column of a 256-byte query row
     const int g0 = 2 * lw + (lane >> 4);          // head row g0 (and g0 + 4 with two loader warps)
-    const int64_t head_stride = static_cast<int64_t>(a.N) * 128;
+    const int64_t head_stride = static_cast<int64_t>(a.Nq) * 128;
     int nq = 0;                        // uses of the query ring so far
     int pend[kLag + 1] = {}, np_head = 0, npend = 0;  // filled stages not yet published (FIFO)
     int4 inf = info(blockIdx.x);
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       const Cursor2 c = cursor(item, inf);
       inf = info(item + gridDim.x);
       const int64_t b = c.bh / a.H_kv, h = c.bh % a.H_kv;
-      const bf16* qg = q + (b * a.H_q + h * 8) * static_cast<int64_t>(a.N) * 128;  // head 0 of the group
+      const bf16* qg = q + (b * a.H_q + h * 8) * head_stride;  // head 0 of the group
       const bf16* qrow0 = qg + g0 * head_stride + jcol * 8;                        // this thread's column of head g0
       for (int tl = 0; tl < c.ntiles; ++tl) {
         const int qs = nq % kQStages;
@@ -260,7 +260,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
       if (lane == 0) mbar_arrive(&accempty[as]);
       ++na;
       int nv = nkeys;
-      if (causal && ok) nv = static_cast<int>(min(static_cast<int64_t>(nv), static_cast<int64_t>(w >> 5) - key0 + 1));
+      if (causal && ok)  // the pair holds the query's row; its position is q0 + row
+        nv = static_cast<int>(min(static_cast<int64_t>(nv), a.q0 + static_cast<int64_t>(w >> 5) - key0 + 1));
       // This warp's columns [kEpiCols hf, kEpiCols (hf + 1)): partial max and
       // sum of exp (four chains each), then the parts of a row are combined.
       const int nvh = nv - kEpiCols * hf;
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         u += __shfl_xor_sync(kFull, u, 2);
         u += __shfl_xor_sync(kFull, u, 4);
         if (ok && (row & 7) == 0) {
-          const int64_t orow = bh * a.N + static_cast<int64_t>(w >> 5);
+          const int64_t orow = bh * a.Nq + static_cast<int64_t>(w >> 5);
           ws.score[orow * 32 + (w & 31)] = u;
         }
       }

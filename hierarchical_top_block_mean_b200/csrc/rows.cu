@@ -21,10 +21,10 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   load_offsets(lay, off);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowWarps + warp;
-  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.N) return;
-  const int64_t bh = row / a.N, t = row % a.N;
+  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.Nq) return;
+  const int64_t bh = row / a.Nq, i = row % a.Nq, t = a.q0 + i;  // query row and its position
   const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
-  stage_q<T, D, G>(q + ((b * a.H_q + h * G) * a.N + t) * D, static_cast<int64_t>(a.N) * D, &qs[warp][0][0]);
+  stage_q<T, D, G>(q + ((b * a.H_q + h * G) * a.Nq + i) * D, static_cast<int64_t>(a.Nq) * D, &qs[warp][0][0]);
   SelectRow<T, D, G> sr{&qs[warp][0][0], pyr + bh * lay.R * D, off, k + bh * a.N * D, a.N, t, a.C, a.K,
                         a.causal != 0, a.scale, tmp[warp]};
   int leaf;
@@ -46,12 +46,12 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   __shared__ int blk[kRowWarps][kMaxK];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowWarps + warp;
-  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.N) return;
-  const int64_t bh = row / a.N, t = row % a.N;
+  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.Nq) return;
+  const int64_t bh = row / a.Nq, i = row % a.Nq, t = a.q0 + i;  // query row and its position
   const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
-  const int64_t hs = static_cast<int64_t>(a.N) * D;
-  const int64_t q0 = ((b * a.H_q + h * G) * a.N + t) * D;
-  stage_q<T, D, G>(q + q0, hs, &qs[warp][0][0]);
+  const int64_t hs = static_cast<int64_t>(a.Nq) * D;
+  const int64_t qo = ((b * a.H_q + h * G) * a.Nq + i) * D;  // head 0 of the group
+  stage_q<T, D, G>(q + qo, hs, &qs[warp][0][0]);
   if (lane < a.K) blk[warp][lane] = sel[row * a.K + lane];
   __syncwarp();
   AttendRow<T, D, G> ar{&qs[warp][0][0], k + bh * a.N * D, v + bh * a.N * D, a.N, t, a.C, a.causal != 0, a.scale,
@@ -62,8 +62,8 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   for (int g = 0; g < G; ++g) {
     const float inv = l[g] > 0.f ? 1.f / l[g] : 0.f;
 #pragma unroll
-    for (int e = 0; e < kCols; ++e) store_out(out + q0 + g * hs + lane * kCols + e, o[g][e] * inv);
-    if (lse && lane == 0) lse[(b * a.H_q + h * G + g) * a.N + t] = m[g] + logf(l[g]);
+    for (int e = 0; e < kCols; ++e) store_out(out + qo + g * hs + lane * kCols + e, o[g][e] * inv);
+    if (lse && lane == 0) lse[(b * a.H_q + h * G + g) * a.Nq + i] = m[g] + logf(l[g]);
   }
 }
 
@@ -74,17 +74,17 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   __shared__ __align__(16) float qs[kRowWarps][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowWarps + warp;
-  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.N) return;
-  const int64_t bh = row / a.N, t = row % a.N;
+  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.Nq) return;
+  const int64_t bh = row / a.Nq, i = row % a.Nq, t = a.q0 + i;  // query row and its position
   const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
-  const int64_t hs = static_cast<int64_t>(a.N) * D;
-  const T* q0 = q + ((b * a.H_q + h * G) * a.N + t) * D;
+  const int64_t hs = static_cast<int64_t>(a.Nq) * D;
+  const T* qg = q + ((b * a.H_q + h * G) * a.Nq + i) * D;
   // The flat score is linear in q, so the group's heads are summed first.
   for (int e = lane * 4; e < D; e += 128) {
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float4 x = load4(q0 + g * hs + e);
+      const float4 x = load4(qg + g * hs + e);
       s.x += x.x;
       s.y += x.y;
       s.z += x.z;
@@ -132,10 +132,10 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   __shared__ __align__(16) float qs[kRowWarps][G][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowWarps + warp;
-  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.N) return;
-  const int64_t bh = row / a.N, t = row % a.N;
+  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.Nq) return;
+  const int64_t bh = row / a.Nq, i = row % a.Nq, t = a.q0 + i;  // query row and its position
   const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
-  stage_q<T, D, G>(q + ((b * a.H_q + h * G) * a.N + t) * D, static_cast<int64_t>(a.N) * D, &qs[warp][0][0]);
+  stage_q<T, D, G>(q + ((b * a.H_q + h * G) * a.Nq + i) * D, static_cast<int64_t>(a.Nq) * D, &qs[warp][0][0]);
   SelectRow<T, D, G> sr{&qs[warp][0][0], nullptr, nullptr, k + bh * a.N * D, a.N, t, a.C, a.K,
                         a.causal != 0, a.scale, nullptr};
   const int64_t nv = valid_count(a.N, a.C, 1, t, a.causal != 0);
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kRowWarps * 32)
 }
 
 inline unsigned row_blocks(const PrefillArgs& a) {
-  return static_cast<unsigned>((static_cast<int64_t>(a.B) * a.H_kv * a.N + kRowWarps - 1) / kRowWarps);
+  return static_cast<unsigned>((static_cast<int64_t>(a.B) * a.H_kv * a.Nq + kRowWarps - 1) / kRowWarps);
 }
 
 }  // namespace

@@ -49,9 +49,9 @@ inline int window_shift(const PrefillArgs& a) {
 inline size_t al(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 size_t carve(const PrefillArgs& a, char* base, Ws* w) {
-  const size_t rows = static_cast<size_t>(a.B) * a.H_kv * a.N;
+  const size_t rows = static_cast<size_t>(a.B) * a.H_kv * a.Nq;
   const int sh = window_shift(a);
-  const int nwin = static_cast<int>((static_cast<int64_t>(a.N) + (int64_t{1} << sh) - 1) >> sh);
+  const int nwin = static_cast<int>((static_cast<int64_t>(a.Nq) + (int64_t{1} << sh) - 1) >> sh);
   const size_t nb = static_cast<size_t>(a.B) * a.H_kv * nwin * level_size(a.N, a.C, 1);
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -110,9 +110,9 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRouterWarps + warp;
-  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.N) return;
+  if (row >= static_cast<int64_t>(a.B) * a.H_kv * a.Nq) return;
   const int64_t n = a.N;
-  const int64_t bh = row / n, t = row % n;
+  const int64_t bh = row / a.Nq, i_row = row % a.Nq, t = a.q0 + i_row;  // query row and its position
   const int64_t b = bh / a.H_kv, h = bh % a.H_kv;
   const bool causal = a.causal != 0;
   const int C = a.C, K = a.K;
@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
     // Query heads of the group as the B operand (columns = heads, zero padded to 8).
     uint32_t qb[D / 16][2];
     const int hd = gid < G ? gid : G - 1;
-    const bf16* qrow = q + ((b * a.H_q + h * G + hd) * n + t) * D + 4 * tig;
+    const bf16* qrow = q + ((b * a.H_q + h * G + hd) * a.Nq + i_row) * D + 4 * tig;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       const uint2 u = *reinterpret_cast<const uint2*>(qrow + 16 * ks);
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
   }
   ws.cand[row * 32 + lane] = lane < nc ? cand : -1;
   if (lane == 0) ws.ncand[row] = nc;
-  if (lane < nc) atomicAdd(&ws.count[(bh * ws.nwin + (t >> ws.win_shift)) * level_size(n, C, 1) + cand], 1);
+  if (lane < nc) atomicAdd(&ws.count[(bh * ws.nwin + (i_row >> ws.win_shift)) * level_size(n, C, 1) + cand], 1);
 }
 
 // ---------------------------------------------------------------- grouping
@@ -295,8 +295,9 @@ __global__ void __launch_bounds__(1024) scan_kernel(Ws ws, int nb) {
   }
 }
 
-// One thread per (row, slot): writes each pair into its leaf's bucket.
-__global__ void __launch_bounds__(256) scatter_kernel(Ws ws, int64_t rows, int N, int M1) {
+// One thread per (row, slot): writes each pair into its leaf's bucket. A
+// pair holds the query's row index within its (b, kv head), not its position.
+__global__ void __launch_bounds__(256) scatter_kernel(Ws ws, int64_t rows, int Nq, int M1) {
   const int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t row = x >> 5;
   const int slot = static_cast<int>(x & 31);
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ws ws, int64_t rows, int N
   const int nc = ws.ncand[row];
   if (slot >= nc) return;
   const int leaf = ws.cand[row * 32 + slot];
-  const int64_t bh = row / N, t = row % N;
+  const int64_t bh = row / Nq, t = row % Nq;
   const int64_t bucket = (bh * ws.nwin + (t >> ws.win_shift)) * M1 + leaf;
   const int pos = atomicAdd(&ws.fill[bucket], 1);
   ws.pairs[ws.bucket_off[bucket] + pos] = (static_cast<uint32_t>(t) << 5) | static_cast<uint32_t>(slot);
@@ -446,7 +447,7 @@ __global__ void __launch_bounds__(kLeafThreads, 2)
         const int pi = r / G;
         const uint32_t w = __shfl_sync(kFull, pw, pi < kP ? pi : 0);
         ok[half] = pi < kP && w != 0xffffffffu;
-        const int64_t tq = ok[half] ? static_cast<int64_t>(w >> 5) : 0;
+        const int64_t tq = ok[half] ? a.q0 + static_cast<int64_t>(w >> 5) : 0;  // query position
         int64_t nv = nkeys;
         if (causal) nv = min(nv, tq - key0 + 1);
         nvk[half] = static_cast<int>(max(nv, static_cast<int64_t>(0)));
@@ -519,7 +520,7 @@ __global__ void __launch_bounds__(kLeafThreads, 2)
         const int pi = r / G;
         const uint32_t w = __shfl_sync(kFull, pw, pi < kP ? pi : 0);
         if (tig == 0 && (gid % G) == 0 && ok[half]) {
-          const int64_t orow = bh * a.N + static_cast<int64_t>(w >> 5);
+          const int64_t orow = bh * a.Nq + static_cast<int64_t>(w >> 5);
           ws.score[orow * 32 + (w & 31)] = uu;
         }
       }
@@ -574,7 +575,7 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
                            int32_t* sel, float* sel_score, void* ws_ptr, cudaStream_t st) {
   Ws ws;
   carve(a, static_cast<char*>(ws_ptr), &ws);
-  const int64_t rows = static_cast<int64_t>(a.B) * a.H_kv * a.N;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.H_kv * a.Nq;
   const int M1 = static_cast<int>(level_size(a.N, a.C, 1));
   const int nb = a.B * a.H_kv * ws.nwin * M1;
   cudaError_t e = cudaMemsetAsync(ws.count, 0, static_cast<size_t>(nb) * 4, st);
@@ -599,7 +600,7 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   if (e != cudaSuccess) return e;
   scan_kernel<<<1, 1024, 0, st>>>(ws, nb);
   count_launch();
-  scatter_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(ws, rows, a.N, M1);
+  scatter_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(ws, rows, a.Nq, M1);
   count_launch();
   itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(ws, nb, M1);
   count_launch();
@@ -608,7 +609,7 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   } else {
     CUtensorMap tmq, tmk;
     const int G0 = a.H_q / a.H_kv;
-    e = make_tmap_bf16_3d(&tmq, q, a.d, a.N, static_cast<uint64_t>(a.B) * a.H_q, 1, G0);
+    e = make_tmap_bf16_3d(&tmq, q, a.d, a.Nq, static_cast<uint64_t>(a.B) * a.H_q, 1, G0);
     if (e == cudaSuccess) e = make_tmap_bf16_2d(&tmk, k, a.d, static_cast<uint64_t>(a.B) * a.H_kv * a.N, a.C);
     if (e != cudaSuccess) return e;
     unsigned long long* faults = wait_fault_counter();

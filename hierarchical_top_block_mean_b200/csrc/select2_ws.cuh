@@ -14,11 +14,11 @@ struct Ws {
   int32_t* fill;        // [buckets] scatter cursors
   int32_t* bucket_off;  // [buckets + 1] exclusive scan of count
   int32_t* item_off;    // [buckets + 1] exclusive scan of ceil(count / kPairsPerItem)
-  uint32_t* pairs;      // [rows * 32] (t << 5 | slot), grouped by bucket
+  uint32_t* pairs;      // [rows * 32] (query row << 5 | slot), grouped by bucket
   uint4* planes;        // [B*H_kv][R][D/4] pyramid rows as bf16 hi/lo: {hi x4, lo x4} per 4 elements
   int32_t* item_bucket; // [items] bucket of each stage-2 work item
   int4* item_info;      // [items] {b * H_kv + h, first pair, end pair, leaf} of each work item
-  int win_shift;        // queries are bucketed by window t >> win_shift
+  int win_shift;        // query rows are bucketed by window (row >> win_shift)
   int nwin;             // windows per (b, kv head)
 };
 

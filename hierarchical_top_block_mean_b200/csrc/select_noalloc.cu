@@ -59,7 +59,8 @@ extern "C" pisa_status pisa_select_noalloc(const pisa_config* cfg, const void* q
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!q || !k || !pyr || !sel || !al16(q) || !al16(k) || !al16(pyr) || !al16(sel))
     return PISA_ERR_INVALID_ARGUMENT;
-  PrefillArgs a{cfg->B, cfg->N, cfg->H_q, cfg->H_kv, cfg->d, cfg->C, cfg->K, cfg->causal, cfg->dtype, cfg->scale};
+  PrefillArgs a{cfg->B, cfg->N, cfg->H_q, cfg->H_kv, cfg->d, cfg->C, cfg->K, cfg->causal, cfg->dtype, cfg->scale,
+                0, cfg->N};
   if (!(a.scale > 0.f)) a.scale = 1.0f / sqrtf(static_cast<float>(cfg->d));
   if (select2_workspace_bytes(a) > kScratchBytes) return PISA_ERR_WORKSPACE;
   void* scratch = nullptr;

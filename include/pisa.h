@@ -219,6 +219,40 @@ pisa_status pisa_sparse_attn_bwd(const pisa_config* cfg, const void* q, const vo
                                  const int32_t* sel, const void* out, const float* lse, const void* dout, float* dq,
                                  float* dk, float* dv, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------ query shards
+ * Sequence-parallel prefill. Split one sequence's queries by position over
+ * several GPUs, so that each GPU computes only its own rows' selection and
+ * attention. Each query row's selection and attention depend only on that
+ * row and on the keys (§TopK, §BSA), so a shard gives bit-for-bit the rows
+ * that the whole-sequence call gives. The keys, the values and the pyramid
+ * are the whole sequence's; every GPU holds a full copy of them, and the
+ * caller gathers them, for instance with an NCCL all-gather of the
+ * per-GPU key and value slices.
+ *
+ * A shard covers query positions [q0, q0 + n_q) of the N-token sequence that
+ * cfg describes (0 <= q0, 1 <= n_q, q0 + n_q <= N; else
+ * PISA_ERR_INVALID_ARGUMENT). These arrays hold the shard's rows only:
+ *   q         : [B, H_q, n_q, d];  out : [B, H_q, n_q, d];  lse : [B, H_q, n_q]
+ *   sel       : [B, H_kv, n_q, K];  sel_score : [B, H_kv, n_q, K]
+ * These arrays hold all N positions, as in the whole-sequence calls:
+ *   k, v : [B, H_kv, N, d];  pyr : from pisa_build_pyramid over all N keys.
+ * Row j of a shard is the query at position q0 + j. It sees keys <= q0 + j
+ * when causal, and all N keys otherwise. Other arguments, error codes and
+ * ownership are those of pisa_select and pisa_sparse_attn_fwd;
+ * {q0 = 0, n_q = N} is exactly those calls.
+ */
+typedef struct {
+  int32_t q0, n_q;
+} pisa_query_span;
+
+size_t pisa_select_span_workspace_bytes(const pisa_config* cfg, const pisa_query_span* span);
+pisa_status pisa_select_span(const pisa_config* cfg, const pisa_query_span* span, const void* q, const void* k,
+                             const float* pyr, int32_t* sel, float* sel_score, void* ws, size_t ws_bytes,
+                             void* stream);
+pisa_status pisa_sparse_attn_fwd_span(const pisa_config* cfg, const pisa_query_span* span, const void* q,
+                                      const void* k, const void* v, const int32_t* sel, void* out, float* lse,
+                                      void* stream);
+
 /* ---------------------------------------------------------------- decode
  * §Kernels, decoding: the mean pyramid is cached; per new token only the
  * current leaf mean and its ancestor path are updated, and one fused kernel

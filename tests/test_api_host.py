@@ -124,3 +124,29 @@ def test_decode_workspace_size():
     # A needed workspace that is missing is refused before anything is enqueued.
     assert lib.pisa_decode_step(ctypes.byref(bf), ok, ok, ok, ok, ok, ok, ok, None, ok, None, ok, None, None) == 3
     assert lib.pisa_decode_attn(ctypes.byref(bf), ok, ok, ok, ok, ok, ok, None, None, None) == 3
+
+
+def test_query_span_validation():
+    """A query shard must lie inside the sequence; a bad span is refused before
+    anything is enqueued, and a whole-sequence span is the plain call."""
+    lib = _lib.lib()
+    before = lib.pisa_launch_count()
+    cfg = _cfg(N=1000, dtype=1)
+    ok = ctypes.c_void_p(256)
+    whole = _lib.QuerySpan(0, 1000)
+    assert lib.pisa_select_span_workspace_bytes(ctypes.byref(cfg), ctypes.byref(whole)) == \
+        lib.pisa_select_workspace_bytes(ctypes.byref(cfg))
+    part = _lib.QuerySpan(500, 250)
+    need = lib.pisa_select_span_workspace_bytes(ctypes.byref(cfg), ctypes.byref(part))
+    assert 0 < need < lib.pisa_select_workspace_bytes(ctypes.byref(cfg))
+    for q0, n_q in ((-1, 10), (0, 0), (990, 11), (1000, 1), (0, 1001)):
+        sp = _lib.QuerySpan(q0, n_q)
+        assert lib.pisa_select_span_workspace_bytes(ctypes.byref(cfg), ctypes.byref(sp)) == 0
+        assert lib.pisa_select_span(ctypes.byref(cfg), ctypes.byref(sp), ok, ok, ok, ok, None, ok, 1 << 30,
+                                    None) == 1
+        assert lib.pisa_sparse_attn_fwd_span(ctypes.byref(cfg), ctypes.byref(sp), ok, ok, ok, ok, ok, None,
+                                             None) == 1
+    assert lib.pisa_select_span(ctypes.byref(cfg), None, ok, ok, ok, ok, None, ok, 1 << 30, None) == 1
+    assert lib.pisa_sparse_attn_fwd_span(ctypes.byref(cfg), None, ok, ok, ok, ok, ok, None, None) == 1
+    assert lib.pisa_select_span(ctypes.byref(cfg), ctypes.byref(part), ok, ok, ok, ok, None, ok, need - 1, None) == 3
+    assert lib.pisa_launch_count() == before
