@@ -61,22 +61,30 @@ class SeqParallelPrefill:
     Holds the full key and value buffers and this rank's shard (pyramid,
     selection, output and lse rows, workspace), all allocated once. Call it
     with this rank's slices q, k, v [B, H, n, d]. It returns (out [B, H_q, n,
-    d], lse [B, H_q, n], sel [B, H_kv, n, K]) for query positions [q0, q0 + n)."""
+    d], lse [B, H_q, n], sel [B, H_kv, n, K]) for query positions [q0, q0 + n).
 
-    def __init__(self, pr: Problem, group=None, device="cuda"):
+    `shard` replaces the per-rank compute; by default it is a PrefillShard
+    (the CUDA kernels) for this rank's span. Anything with pyramid(k),
+    select(q, k), attend(q, k, v) and out, lse, sel attributes will do."""
+
+    def __init__(self, pr: Problem, group=None, device="cuda", shard=None):
         self.pr, self.group = pr, group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.q0, self.n = shard_span(pr.N, self.world, self.rank)
         dev = torch.device(device)
-        self.shard = PrefillShard(pr, self.q0, self.n, dev)
+        self._kernels = shard is None  # the default shard runs the library's CUDA kernels
+        self.shard = PrefillShard(pr, self.q0, self.n, dev) if shard is None else shard
         self.k_full = torch.empty((pr.B, pr.H_kv, pr.N, pr.d), dtype=pr.dtype, device=dev)
         self.v_full = torch.empty_like(self.k_full)
 
     def _check(self, q, k, v):
         pr = self.pr
         for t, name, H in ((q, "q", pr.H_q), (k, "k", pr.H_kv), (v, "v", pr.H_kv)):
-            _need(t, name, pr.dtype)
+            if self._kernels:
+                _need(t, name, pr.dtype)
+            elif t.dtype != pr.dtype or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous {pr.dtype} tensor")
             if tuple(t.shape) != (pr.B, H, self.n, pr.d):
                 raise ValueError(f"{name} {tuple(t.shape)} is not this rank's slice [{pr.B}, {H}, {self.n}, {pr.d}]")
 
