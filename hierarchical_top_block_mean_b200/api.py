@@ -312,6 +312,73 @@ def prefill(q, k, v, *, C: int, K: int, causal: bool, scale: float = 0.0):
     return p.out, p.lse, p.sel
 
 
+class PrefillStream:
+    """Prefill steps over batches held in pinned host memory, with the
+    host-device copies overlapped with compute.
+
+    While step s computes on the current stream, step s + 1's q, k and v are
+    copied in on one copy stream, and step s - 1's output is copied out on
+    another. Each step uses one of `depth` slots: device inputs plus a
+    Prefill pipeline with its own outputs. Events order the slots, so a slot
+    is refilled only after its previous step has computed, and recomputed
+    only after its previous output has been copied out.
+
+    The host tensors passed to submit() must stay alive and unchanged until
+    that step's output copy has finished (synchronize(), or the returned
+    event)."""
+
+    def __init__(self, pr: Problem, device="cuda", depth: int = 2):
+        if depth < 1:
+            raise ValueError("depth must be at least 1")
+        dev = torch.device(device)
+        self.pr, self.dev = pr, dev
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.slots = []
+        for _ in range(depth):
+            self.slots.append({
+                "p": Prefill(pr, dev),
+                "q": torch.empty((pr.B, pr.H_q, pr.N, pr.d), dtype=pr.dtype, device=dev),
+                "k": torch.empty((pr.B, pr.H_kv, pr.N, pr.d), dtype=pr.dtype, device=dev),
+                "v": torch.empty((pr.B, pr.H_kv, pr.N, pr.d), dtype=pr.dtype, device=dev),
+                "loaded": torch.cuda.Event(), "computed": torch.cuda.Event(), "drained": torch.cuda.Event(),
+            })
+        self.steps = 0
+
+    def submit(self, hq, hk, hv, hout):
+        """Enqueues one step: hq, hk, hv (pinned host [B, H, N, d]) in, the
+        prefill, its output into hout (pinned host [B, H_q, N, d]). Returns
+        the event that completes when hout holds the output."""
+        pr = self.pr
+        for t, name, H in ((hq, "q", pr.H_q), (hk, "k", pr.H_kv), (hv, "v", pr.H_kv), (hout, "out", pr.H_q)):
+            if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous tensor in pinned host memory")
+            if t.dtype != pr.dtype or tuple(t.shape) != (pr.B, H, pr.N, pr.d):
+                raise ValueError(f"{name} must be {pr.dtype} [{pr.B}, {H}, {pr.N}, {pr.d}]")
+        slot = self.slots[self.steps % len(self.slots)]
+        self.steps += 1
+        compute = torch.cuda.current_stream(self.dev)
+        self.h2d.wait_event(slot["computed"])  # the slot's previous step has read its inputs
+        with torch.cuda.stream(self.h2d):
+            slot["q"].copy_(hq, non_blocking=True)
+            slot["k"].copy_(hk, non_blocking=True)
+            slot["v"].copy_(hv, non_blocking=True)
+            slot["loaded"].record(self.h2d)
+        compute.wait_event(slot["loaded"])
+        compute.wait_event(slot["drained"])  # the slot's previous output has been copied out
+        slot["p"](slot["q"], slot["k"], slot["v"])
+        slot["computed"].record(compute)
+        self.d2h.wait_event(slot["computed"])
+        with torch.cuda.stream(self.d2h):
+            hout.copy_(slot["p"].out, non_blocking=True)
+            slot["drained"].record(self.d2h)
+        return slot["drained"]
+
+    def synchronize(self):
+        """Waits on the host until every submitted step's output is in host memory."""
+        self.d2h.synchronize()
+
+
 class DecodeState:
     """Caller-side decode state for S sequences of capacity cap: KV caches,
     the cached mean pyramid, per-sequence lengths, a device status word and
