@@ -1,7 +1,9 @@
 /*
  * pisa.h — C ABI of the B200 (sm_100a) PISA hot path: mean-pooled key
- * pyramid, coarse-to-fine top-K block selection, flat single-level block
- * selection, block-sparse attention forward, and the decode step.
+ * pyramid, coarse-to-fine top-K block selection, flat and exact-score
+ * single-level block selection, block-sparse attention forward and backward,
+ * query shards for sequence-parallel prefill, and the decode step over dense
+ * or paged KV caches.
  *
  * The method is "Block Sparse Attention with Log-Linear Complexity"
  * (Tang, Qin, Pan, Li, Liu). Citations below name sections of its hyper.ai
@@ -245,6 +247,8 @@ typedef struct {
   int32_t q0, n_q;
 } pisa_query_span;
 
+/* Scratch bytes pisa_select_span needs: it scales with n_q, not N. Returns
+ * 0 for an invalid cfg or span, and for fp32, which needs none. */
 size_t pisa_select_span_workspace_bytes(const pisa_config* cfg, const pisa_query_span* span);
 pisa_status pisa_select_span(const pisa_config* cfg, const pisa_query_span* span, const void* q, const void* k,
                              const float* pyr, int32_t* sel, float* sel_score, void* ws, size_t ws_bytes,
