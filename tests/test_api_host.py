@@ -150,3 +150,21 @@ def test_query_span_validation():
     assert lib.pisa_sparse_attn_fwd_span(ctypes.byref(cfg), None, ok, ok, ok, ok, ok, None, None) == 1
     assert lib.pisa_select_span(ctypes.byref(cfg), ctypes.byref(part), ok, ok, ok, ok, None, ok, need - 1, None) == 3
     assert lib.pisa_launch_count() == before
+
+
+def test_header_compiles_as_c99_and_links(tmp_path):
+    """The boundary is a C ABI: a plain C99 program includes pisa.h, links the
+    library and runs its host-only calls (no GPU needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    exe = str(tmp_path / "abi_check")
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_check.c"), "-L", lib_dir, "-lpisa_b200",
+                    "-Wl,-rpath," + lib_dir, "-o", exe], check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "FAIL" not in r.stdout and r.stdout.count("ok ") == 13, r.stdout
