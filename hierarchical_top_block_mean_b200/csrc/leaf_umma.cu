@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         // Loader thread (warp lw, lane l): 16-byte column j = l & 15 of head
         // row g0 = 2 lw + (l >> 4) (and g0 + 4 with two loader warps) of every query of the tile,
         // so each copy instruction moves two whole 256-byte rows. The tile's
-        // query positions are read once per warp and shared by shuffle.
+        // query rows are read once per warp and shared by shuffle.
         const int tw = lane < np ? static_cast<int>(ws.pairs[p0 + lane] >> 5) : 0;
         mbar_wait(&qempty[qs], ((nq / kQStages) & 1) ^ 1, faults);
         const uint32_t qd = smem_u32(qbuf + qs * kQStageBytes);
