@@ -240,6 +240,47 @@ def cpu_baseline(w, x, budget_s=15.0):
                       f"(kv head, query) rows ({t_rows:.1f} s), extrapolated linearly to all {total_rows} rows"}
 
 
+def cpu_decode_baseline(wd, budget_s=5.0):
+    """The fp64 CPU oracle as it stands, on a bounded sample of the decode
+    step. The sample is one sequence at the workload's context length with
+    all its kv heads, timed per step for the append's pyramid update (per
+    head), the root-to-leaf selection and the attention of the new token (all
+    heads' rows in one call each, which the oracle spreads over its threads).
+    The prefix pyramid is the cached state and is built untimed. The result
+    is scaled linearly to all S sequences."""
+    import numpy as np
+    import oracle as O
+    O.build()
+    cores = len(os.sched_getaffinity(0))
+    n = wd.context + 1  # tokens held once the step's token is appended
+    cfg = O.make_cfg(B=1, N=n, H_q=wd.H_q, H_kv=wd.H_kv, d=wd.d, C=wd.C, K=wd.K, causal=True, dtype_code=1,
+                     Nq=1, q_t0=n - 1)
+    _, offs_c = O.geometry(wd.cap, wd.C)
+    g = torch.Generator().manual_seed(wd.seed + 77)
+    # One sequence's cache serves every timed step: the work does not depend
+    # on the cached values, and each step draws its own query.
+    k = torch.randn(1, wd.H_kv, n, wd.d, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, wd.H_kv, n, wd.d, generator=g).to(torch.bfloat16)
+    pyr = O.build_pyramid(k, wd.C)
+    cap_pyr = [np.zeros((offs_c[-1], wd.d), np.float64) for _ in range(wd.H_kv)]
+    rows = [(0, h, n - 1) for h in range(wd.H_kv)]
+    t_step, seqs = 0.0, 0
+    while seqs < wd.S and (seqs == 0 or t_step < budget_s):
+        q = torch.randn(1, wd.H_q, 1, wd.d, generator=g).to(torch.bfloat16)
+        t0 = time.perf_counter()
+        for h in range(wd.H_kv):
+            O.decode_append(k[0, h], n - 1, wd.C, wd.cap, cap_pyr[h])
+        sel, _ = O.select_rows(cfg, q, k, pyr, rows)
+        O.attn_rows(cfg, q, k, v, rows, sel)
+        t_step += time.perf_counter() - t0
+        seqs += 1
+    us = t_step / seqs * wd.S * 1e6
+    return {"us_per_step": us, "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle: append + select + attention of the new token for {seqs} steps of one "
+                      f"sequence ({wd.H_kv} kv heads) at {n} tokens ({t_step:.2f} s), extrapolated linearly "
+                      f"to {wd.S} sequences; {wd.H_kv} rows per oracle call"}
+
+
 def run_reference(args):
     """Reference arm: the CPU oracle as it stands, timed on the host cores.
     Under torchrun only rank 0 runs it; the other ranks exit without work
@@ -510,6 +551,8 @@ def run_gpu(args):
         torch.cuda.empty_cache()
         decode = time_decode(workloads.DECODE[args.decode_workload])
         decode["paged"] = time_decode_paged(workloads.DECODE[args.decode_workload])
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            decode["cpu_baseline"] = cpu_decode_baseline(workloads.DECODE[args.decode_workload])
 
     pk, pk_kind = peaks()
     # Roofline of the dominant stage (the attention kernel: one launch per step).

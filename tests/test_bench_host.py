@@ -43,3 +43,14 @@ def test_traffic_record_is_dropped_when_a_source_changes(tmp_path, monkeypatch):
     src.write_text("kernel v2")
     assert bench.measured_traffic("w", "attn") is None
     assert bench.measured_traffic("other", "attn") is None
+
+
+def test_cpu_decode_baseline_on_a_small_decode_workload():
+    """The decode CPU baseline runs the oracle's append, selection and
+    attention for a whole step's sequences when they fit the budget, and
+    labels what it timed."""
+    from hierarchical_top_block_mean_b200 import workloads
+    wd = workloads.DECODE["decode_64x128k"].with_(name="dec_tiny", S=3, context=700, H_q=8, H_kv=2)
+    r = bench.cpu_decode_baseline(wd, budget_s=1.0)
+    assert r["kind"] == "oracle" and r["us_per_step"] > 0 and r["cores"] >= 1
+    assert "3 steps" in r["sample"] and "701 tokens" in r["sample"]
