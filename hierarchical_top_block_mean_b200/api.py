@@ -26,15 +26,23 @@ def _stream(t: torch.Tensor):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
-def _need(t: torch.Tensor, name: str, dtype=None):
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
+    """Checks a tensor handed to the library: the kernels trust every size, so
+    a buffer of the wrong shape would be read or written out of bounds."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    _on_cuda(t, name)
+
+
+def _on_cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
 
 
 def launch_count() -> int:
@@ -105,7 +113,7 @@ def build_pyramid(k: torch.Tensor, *, C: int, out: torch.Tensor | None = None) -
     pr = Problem(B, N, H, H, d, C, 1, False, k.dtype)
     if out is None:
         out = torch.empty((B, H, pr.R, d), dtype=torch.float32, device=k.device)
-    _need(out, "out", torch.float32)
+    _need(out, "out", torch.float32, (B, H, pr.R, d))
     _lib.call("pisa_build_pyramid", ctypes.byref(pr.cstruct()), _p(k), _p(out), _stream(k))
     return out
 
@@ -113,14 +121,20 @@ def build_pyramid(k: torch.Tensor, *, C: int, out: torch.Tensor | None = None) -
 def select(q, k, pyr, *, C: int, K: int, causal: bool, scale: float = 0.0, out=None, score=None,
            workspace=None):
     """PISA coarse-to-fine top-K leaf blocks: sel [B, H_kv, N, K] int32 (ascending, -1 padded)."""
-    for t, n in ((q, "q"), (k, "k"), (pyr, "pyr")):
-        _need(t, n)
+    _need(q, "q")
+    _need(k, "k", q.dtype)
     pr = Problem.of(q, k, C=C, K=K, causal=causal, scale=scale)
+    _need(pyr, "pyr", torch.float32, (pr.B, pr.H_kv, pr.R, pr.d))
+    rows = (pr.B, pr.H_kv, pr.N, K)
     if out is None:
-        out = torch.empty((pr.B, pr.H_kv, pr.N, K), dtype=torch.int32, device=q.device)
+        out = torch.empty(rows, dtype=torch.int32, device=q.device)
+    _need(out, "out", torch.int32, rows)
+    if score is not None:
+        _need(score, "score", torch.float32, rows)
     need = pr.workspace_bytes()
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
     _lib.call("pisa_select", ctypes.byref(pr.cstruct()), _p(q), _p(k), _p(pyr), _p(out), _p(score), _p(workspace),
               workspace.numel() * workspace.element_size(), _stream(q))
     return out
@@ -129,11 +143,12 @@ def select(q, k, pyr, *, C: int, K: int, causal: bool, scale: float = 0.0, out=N
 def select_flat(q, pyr, *, C: int, K: int, causal: bool, H_kv: int, scale: float = 0.0, out=None):
     """Flat single-level top-K over all leaf summaries: sel [B, H_kv, N, K] int32."""
     _need(q, "q")
-    _need(pyr, "pyr", torch.float32)
     B, H_q, N, d = q.shape
     pr = Problem(B, N, H_q, H_kv, d, C, K, bool(causal), q.dtype, scale)
+    _need(pyr, "pyr", torch.float32, (B, H_kv, pr.R, d))
     if out is None:
         out = torch.empty((B, H_kv, N, K), dtype=torch.int32, device=q.device)
+    _need(out, "out", torch.int32, (B, H_kv, N, K))
     _lib.call("pisa_select_flat", ctypes.byref(pr.cstruct()), _p(q), _p(pyr), _p(out), _stream(q))
     return out
 
@@ -142,11 +157,14 @@ def sparse_attn_bwd(q, k, v, sel, out, lse, dout, *, C: int, causal: bool, scale
     """Gradients (dq, dk, dv; fp32) of the block-sparse attention with the
     selection sel held fixed, for the output gradient dout; out and lse are the
     forward's outputs. bf16 inputs."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
-        _need(t, n, q.dtype)
-    _need(sel, "sel", torch.int32)
-    _need(lse, "lse", torch.float32)
+    _need(q, "q")
+    _need(k, "k", q.dtype)
+    _need(v, "v", q.dtype, k.shape)
+    _need(out, "out", q.dtype, q.shape)
+    _need(dout, "dout", q.dtype, q.shape)
     pr = Problem.of(q, k, C=C, K=sel.shape[-1], causal=causal, scale=scale)
+    _need(sel, "sel", torch.int32, (pr.B, pr.H_kv, pr.N, pr.K))
+    _need(lse, "lse", torch.float32, (pr.B, pr.H_q, pr.N))
     cfg = pr.cstruct()
     nbytes = int(_lib.lib().pisa_attn_bwd_workspace_bytes(ctypes.byref(cfg)))
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
@@ -166,6 +184,7 @@ def select_exact(q, k, *, C: int, K: int, causal: bool, scale: float = 0.0, out=
     pr = Problem.of(q, k, C=C, K=K, causal=causal, scale=scale)
     if out is None:
         out = torch.empty((pr.B, pr.H_kv, pr.N, K), dtype=torch.int32, device=q.device)
+    _need(out, "out", torch.int32, (pr.B, pr.H_kv, pr.N, K))
     _lib.call("pisa_select_exact", ctypes.byref(pr.cstruct()), _p(q), _p(k), _p(out), _stream(q))
     return out
 
@@ -173,15 +192,18 @@ def select_exact(q, k, *, C: int, K: int, causal: bool, scale: float = 0.0, out=
 def sparse_attn_fwd(q, k, v, sel, *, C: int, causal: bool, scale: float = 0.0, out=None, lse=None,
                     want_lse: bool = True):
     """Block-sparse attention over the selected leaf blocks: (out [B,H_q,N,d], lse [B,H_q,N] or None)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n)
-    _need(sel, "sel", torch.int32)
-    K = sel.shape[-1]
-    pr = Problem.of(q, k, C=C, K=K, causal=causal, scale=scale)
+    _need(q, "q")
+    _need(k, "k", q.dtype)
+    _need(v, "v", q.dtype, k.shape)
+    pr = Problem.of(q, k, C=C, K=sel.shape[-1], causal=causal, scale=scale)
+    _need(sel, "sel", torch.int32, (pr.B, pr.H_kv, pr.N, pr.K))
     if out is None:
         out = torch.empty_like(q)
+    _need(out, "out", q.dtype, q.shape)
     if lse is None and want_lse:
         lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, q.shape[:-1])
     _lib.call("pisa_sparse_attn_fwd", ctypes.byref(pr.cstruct()), _p(q), _p(k), _p(v), _p(sel), _p(out), _p(lse),
               _stream(q))
     return out, lse
@@ -201,15 +223,21 @@ def select_span(q, k, pyr, *, q0: int, C: int, K: int, causal: bool, scale: floa
     q [B, H_q, n_q, d] holds those rows only; k [B, H_kv, N, d] and pyr cover
     all N tokens. Returns sel [B, H_kv, n_q, K], equal to those rows of a
     whole-sequence selection."""
-    for t, n in ((q, "q"), (k, "k"), (pyr, "pyr")):
-        _need(t, n)
+    _need(q, "q")
+    _need(k, "k", q.dtype)
     pr, n_q = _span_problem(q, k, C, K, causal, scale)
+    _need(pyr, "pyr", torch.float32, (pr.B, pr.H_kv, pr.R, pr.d))
     cfg, span = pr.cstruct(), _lib.QuerySpan(q0, n_q)
+    rows = (pr.B, pr.H_kv, n_q, K)
     if out is None:
-        out = torch.empty((pr.B, pr.H_kv, n_q, K), dtype=torch.int32, device=q.device)
+        out = torch.empty(rows, dtype=torch.int32, device=q.device)
+    _need(out, "out", torch.int32, rows)
+    if score is not None:
+        _need(score, "score", torch.float32, rows)
     if workspace is None:
         need = int(_lib.lib().pisa_select_span_workspace_bytes(ctypes.byref(cfg), ctypes.byref(span)))
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
     _lib.call("pisa_select_span", ctypes.byref(cfg), ctypes.byref(span), _p(q), _p(k), _p(pyr), _p(out), _p(score),
               _p(workspace), workspace.numel() * workspace.element_size(), _stream(q))
     return out
@@ -220,14 +248,18 @@ def sparse_attn_fwd_span(q, k, v, sel, *, q0: int, C: int, causal: bool, scale: 
     """Block-sparse attention for the query rows at positions [q0, q0 + n_q):
     q [B, H_q, n_q, d] and sel [B, H_kv, n_q, K] hold those rows; k and v all
     N tokens. Returns (out [B, H_q, n_q, d], lse [B, H_q, n_q] or None)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n)
-    _need(sel, "sel", torch.int32)
+    _need(q, "q")
+    _need(k, "k", q.dtype)
+    _need(v, "v", q.dtype, k.shape)
     pr, n_q = _span_problem(q, k, C, sel.shape[-1], causal, scale)
+    _need(sel, "sel", torch.int32, (pr.B, pr.H_kv, n_q, pr.K))
     if out is None:
         out = torch.empty_like(q)
+    _need(out, "out", q.dtype, q.shape)
     if lse is None and want_lse:
         lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, q.shape[:-1])
     _lib.call("pisa_sparse_attn_fwd_span", ctypes.byref(pr.cstruct()), ctypes.byref(_lib.QuerySpan(q0, n_q)), _p(q),
               _p(k), _p(v), _p(sel), _p(out), _p(lse), _stream(q))
     return out, lse
@@ -235,7 +267,9 @@ def sparse_attn_fwd_span(q, k, v, sel, *, q0: int, C: int, causal: bool, scale: 
 
 class Prefill:
     """Reusable prefill pipeline for one problem shape: pyramid, PISA select
-    and block-sparse attention, with all buffers allocated once."""
+    and block-sparse attention, with all buffers allocated once. Calling it
+    checks q, k and v against the problem. The stage methods (pyramid,
+    select, attend) skip that check and expect the problem's shapes."""
 
     def __init__(self, pr: Problem, device="cuda"):
         self.pr = pr
@@ -258,7 +292,15 @@ class Prefill:
         _lib.call("pisa_sparse_attn_fwd", ctypes.byref(self.cfg), _p(q), _p(k), _p(v), _p(self.sel), _p(self.out),
                   _p(self.lse), _stream(q))
 
+    def check(self, q, k, v):
+        """Raises unless q, k and v have this problem's shapes and dtype."""
+        pr = self.pr
+        _need(q, "q", pr.dtype, (pr.B, pr.H_q, pr.N, pr.d))
+        _need(k, "k", pr.dtype, (pr.B, pr.H_kv, pr.N, pr.d))
+        _need(v, "v", pr.dtype, (pr.B, pr.H_kv, pr.N, pr.d))
+
     def __call__(self, q, k, v):
+        self.check(q, k, v)
         self.pyramid(k)
         self.select(q, k)
         self.attend(q, k, v)
@@ -269,7 +311,8 @@ class PrefillShard:
     """Prefill of the query rows at positions [q0, q0 + n_q) of an N-token
     sequence (pr describes the whole sequence): the pyramid over all N keys,
     then the selection and attention of this shard's rows only, with buffers
-    allocated once. q is [B, H_q, n_q, d]; k and v are [B, H_kv, N, d]."""
+    allocated once. q is [B, H_q, n_q, d]; k and v are [B, H_kv, N, d].
+    Calling it checks them; the stage methods do not."""
 
     def __init__(self, pr: Problem, q0: int, n_q: int, device="cuda"):
         self.pr, self.q0, self.n_q = pr, q0, n_q
@@ -296,7 +339,15 @@ class PrefillShard:
         _lib.call("pisa_sparse_attn_fwd_span", ctypes.byref(self.cfg), ctypes.byref(self.span), _p(q), _p(k), _p(v),
                   _p(self.sel), _p(self.out), _p(self.lse), _stream(q))
 
+    def check(self, q, k, v):
+        """Raises unless q holds this shard's rows and k, v the whole sequence."""
+        pr = self.pr
+        _need(q, "q", pr.dtype, (pr.B, pr.H_q, self.n_q, pr.d))
+        _need(k, "k", pr.dtype, (pr.B, pr.H_kv, pr.N, pr.d))
+        _need(v, "v", pr.dtype, (pr.B, pr.H_kv, pr.N, pr.d))
+
     def __call__(self, q, k, v):
+        self.check(q, k, v)
         self.pyramid(k)
         self.select(q, k)
         self.attend(q, k, v)
@@ -413,23 +464,34 @@ class DecodeState:
         _lib.call("pisa_decode_init", ctypes.byref(self.cfg), _p(self.k_cache), _p(self.pyr), _p(self.len),
                   _stream(self.pyr))
 
+    def _check_new(self, q_new=None, k_new=None, v_new=None):
+        """Raises unless the step's tensors are [S, H_q, d] (q) and [S, H_kv, d] (k, v) in the cache dtype."""
+        for t, name, H in ((q_new, "q_new", self.H_q), (k_new, "k_new", self.H_kv), (v_new, "v_new", self.H_kv)):
+            if t is not None:
+                _need(t, name, self.dtype, (self.S, H, self.d))
+
     def append(self, k_new, v_new):
+        self._check_new(k_new=k_new, v_new=v_new)
         _lib.call("pisa_decode_append", ctypes.byref(self.cfg), _p(k_new), _p(v_new), _p(self.k_cache),
                   _p(self.v_cache), _p(self.pyr), _p(self.len), _p(self.status), _stream(self.pyr))
 
     def select(self, q_new):
+        self._check_new(q_new=q_new)
         _lib.call("pisa_decode_select", ctypes.byref(self.cfg), _p(q_new), _p(self.k_cache), _p(self.pyr),
                   _p(self.len), _p(self.sel), _stream(self.pyr))
         return self.sel
 
     def attend(self, q_new, sel=None):
+        self._check_new(q_new=q_new)
         s = self.sel if sel is None else sel
+        _need(s, "sel", torch.int32, (self.S, self.H_kv, self.K))
         _lib.call("pisa_decode_attn", ctypes.byref(self.cfg), _p(q_new), _p(self.k_cache), _p(self.v_cache),
                   _p(self.len), _p(s), _p(self.out), _p(self.lse), _p(self.workspace), _stream(self.pyr))
         return self.out
 
     def step(self, q_new, k_new, v_new, keep_sel: bool = True):
         """Append + select + attend for every sequence."""
+        self._check_new(q_new, k_new, v_new)
         _lib.call("pisa_decode_step", ctypes.byref(self.cfg), _p(q_new), _p(k_new), _p(v_new), _p(self.k_cache),
                   _p(self.v_cache), _p(self.pyr), _p(self.len), _p(self.sel) if keep_sel else None, _p(self.out),
                   _p(self.lse), _p(self.status), _p(self.workspace), _stream(self.pyr))
@@ -452,6 +514,7 @@ class PagedDecodeState:
         cap = max_pages * C
         self.cfg = _lib.DecodeConfig(S, cap, H_q, H_kv, d, C, 2, K, _DT[dtype], scale)
         self.S, self.cap, self.max_pages, self.H_q, self.H_kv, self.d, self.C, self.K = S, cap, max_pages, H_q, H_kv, d, C, K
+        self.dtype = dtype
         for t, n in ((k_pages, "k_pages"), (v_pages, "v_pages")):
             _need(t, n, dtype)
         _need(block_table, "block_table", torch.int32)
@@ -478,6 +541,8 @@ class PagedDecodeState:
 
     def step(self, q_new, k_new, v_new, keep_sel: bool = True):
         """Append + select + attend for every sequence."""
+        for t, name, H in ((q_new, "q_new", self.H_q), (k_new, "k_new", self.H_kv), (v_new, "v_new", self.H_kv)):
+            _need(t, name, self.dtype, (self.S, H, self.d))
         _lib.call("pisa_decode_step_paged", ctypes.byref(self.cfg), _p(q_new), _p(k_new), _p(v_new),
                   _p(self.k_pages), _p(self.v_pages), _p(self.block_table), self.max_pages, _p(self.pyr),
                   _p(self.len), _p(self.sel) if keep_sel else None, _p(self.out), _p(self.lse), _p(self.status),
