@@ -515,12 +515,14 @@ class PagedDecodeState:
         self.cfg = _lib.DecodeConfig(S, cap, H_q, H_kv, d, C, 2, K, _DT[dtype], scale)
         self.S, self.cap, self.max_pages, self.H_q, self.H_kv, self.d, self.C, self.K = S, cap, max_pages, H_q, H_kv, d, C, K
         self.dtype = dtype
+        if k_pages.dim() != 4:
+            raise ValueError("k_pages must be [num_pages, H_kv, C, d]")
+        self.num_pages = k_pages.shape[0]
         for t, n in ((k_pages, "k_pages"), (v_pages, "v_pages")):
-            _need(t, n, dtype)
-        _need(block_table, "block_table", torch.int32)
-        _need(lens, "lens", torch.int32)
-        if tuple(block_table.shape) != (S, max_pages):
-            raise ValueError("block_table must be [S, max_pages]")
+            _need(t, n, dtype, (self.num_pages, H_kv, C, d))
+        _need(block_table, "block_table", torch.int32, (S, max_pages))
+        _need(lens, "lens", torch.int32, (S,))
+        self.check_block_table(block_table)
         self.k_pages, self.v_pages, self.block_table, self.len = k_pages, v_pages, block_table, lens
         R = int(_lib.lib().pisa_decode_pyramid_rows(ctypes.byref(self.cfg)))
         if R <= 0:
@@ -533,6 +535,14 @@ class PagedDecodeState:
         self.lse = torch.empty((S, H_q), dtype=torch.float32, device=dev)
         ws = int(_lib.lib().pisa_decode_workspace_bytes(ctypes.byref(self.cfg)))
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+
+    def check_block_table(self, block_table=None):
+        """Raises unless every entry is -1 or a page of the pool. The kernels
+        cannot bound page indices, so call this again after editing the table
+        (it reads the table back to the host, which synchronises)."""
+        bt = self.block_table if block_table is None else block_table
+        if bt.numel() and (int(bt.min()) < -1 or int(bt.max()) >= self.num_pages):
+            raise ValueError(f"block_table entries must be -1 or pages 0..{self.num_pages - 1}")
 
     def init(self):
         """Builds each sequence's pyramid over its first len[s] cached tokens."""

@@ -316,7 +316,11 @@ pisa_status pisa_decode_step(const pisa_decode_config* cfg, const void* q_new, c
  * for every kv head.
  *   k_pages, v_pages : [num_pages, H_kv, C, d] in dtype (bf16 only);
  *   block_table      : [S, max_pages] int32 device; entry i is the page of
- *                      leaf i of the sequence, -1 where none is assigned;
+ *                      leaf i of the sequence, -1 where none is assigned.
+ *                      Every other entry must be a page of the pool
+ *                      (0 <= entry < num_pages): the library does not know
+ *                      num_pages and cannot check it, so an entry out of range
+ *                      makes the kernels read and write outside the pool;
  *   cfg->cap         : must equal max_pages * C.
  * Pages of the leaves a sequence already holds must be assigned. A step whose
  * new token falls in a leaf without a page stores PISA_ERR_CAPACITY in status

@@ -113,3 +113,26 @@ def test_decode_state_checks_step_tensors(calls):
     ps.step(qn, kn, vn)
     assert calls[-1] == "pisa_decode_step_paged"
     _refused(calls, ps.step, qn, kn, vn[:, :, :-1].contiguous())
+
+
+def test_paged_state_refuses_out_of_pool_pages(calls):
+    S, Hq, Hkv, P = 2, 8, 2, 5
+    pages = torch.zeros(P, Hkv, C, d, dtype=bf)
+    lens = torch.zeros(S, dtype=torch.int32)
+
+    def make(bt, kp=pages):
+        return api.PagedDecodeState(S=S, max_pages=3, H_q=Hq, H_kv=Hkv, d=d, C=C, K=K, k_pages=kp, v_pages=kp,
+                                    block_table=bt, lens=lens)
+
+    ok = make(torch.tensor([[0, 1, -1], [2, 3, 4]], dtype=torch.int32))
+    for bad in ([[0, 1, 5], [2, 3, 4]], [[0, -2, 1], [2, 3, 4]]):
+        with pytest.raises(ValueError):
+            make(torch.tensor(bad, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        make(torch.zeros(S, 2, dtype=torch.int32))  # not [S, max_pages]
+    with pytest.raises(ValueError):
+        make(torch.zeros(S, 3, dtype=torch.int32), kp=torch.zeros(P, Hkv, C // 2, d, dtype=bf))
+    ok.block_table[1, 2] = P  # an edit after construction is caught by the explicit check
+    with pytest.raises(ValueError):
+        ok.check_block_table()
+    assert calls == []
