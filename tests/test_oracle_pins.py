@@ -554,3 +554,31 @@ def test_decode_query_sees_every_block(oracle):
     q1 = x["q"][:, :, t:t + 1, :].contiguous()
     s3, _ = oracle.select_rows(_cfg(oracle, w, Nq=1, q_t0=t), q1, x["k"], pyr, rows)
     assert (s1 == s3).all()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_held_query_block_gives_the_whole_sequence_rows(oracle, causal):
+    # A block of query rows held at an unaligned offset (a sequence-parallel
+    # shard, or decode's single row) must give the rows that the whole
+    # sequence's queries give: row j of the block is position q_t0 + j.
+    w = _small(N=600, C=16, K=4, causal=causal, dtype="bf16", seed=91)
+    x = workloads.prefill_inputs(w)
+    pyr = oracle.build_pyramid(x["k"], w.C)
+    a, b = 123, 411
+    rng = np.random.default_rng(5)
+    ts = np.unique(np.concatenate([[a, b - 1], rng.integers(a, b, 40)]))
+    rows = [(0, h, int(t)) for h in range(w.H_kv) for t in ts]
+    s_all, g_all = oracle.select_rows(_cfg(oracle, w), x["q"], x["k"], pyr, rows)
+    qb = x["q"][:, :, a:b].contiguous()
+    cfg_b = _cfg(oracle, w, Nq=b - a, q_t0=a)
+    s_blk, g_blk = oracle.select_rows(cfg_b, qb, x["k"], pyr, rows)
+    assert (s_all == s_blk).all() and np.array_equal(g_all, g_blk)
+    o_all, l_all = oracle.attn_rows(_cfg(oracle, w), x["q"], x["k"], x["v"], rows, s_all)
+    o_blk, l_blk = oracle.attn_rows(cfg_b, qb, x["k"], x["v"], rows, s_all)
+    assert np.array_equal(o_all, o_blk) and np.array_equal(l_all, l_blk)
+    if causal:
+        # The offset matters under the causal reading: the block read as if
+        # it started at position 0 sees fewer blocks and selects differently.
+        s_wrong, _ = oracle.select_rows(_cfg(oracle, w, Nq=b - a, q_t0=0), qb, x["k"], pyr,
+                                        [(0, h, int(t) - a) for h in range(w.H_kv) for t in ts])
+        assert not (s_wrong == s_all).all()
