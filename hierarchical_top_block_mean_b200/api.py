@@ -394,6 +394,13 @@ class PrefillStream:
                 "v": torch.empty((pr.B, pr.H_kv, pr.N, pr.d), dtype=pr.dtype, device=dev),
                 "loaded": torch.cuda.Event(), "computed": torch.cuda.Event(), "drained": torch.cuda.Event(),
             })
+        # The copy streams use these buffers. If this object is dropped with
+        # copies still queued, the allocator must not hand the memory to a
+        # new tensor until they finish.
+        for slot in self.slots:
+            for name in ("q", "k", "v"):
+                slot[name].record_stream(self.h2d)
+            slot["p"].out.record_stream(self.d2h)
         self.steps = 0
 
     def submit(self, hq, hk, hv, hout):
