@@ -1,4 +1,4 @@
-"""Host logic of sequence-parallel prefill on CPU, run as two gloo ranks:
+"""Host logic of sequence-parallel prefill on CPU, run as gloo ranks (two, and four for the gather):
 the shard arithmetic; the all-gather that assembles every rank's key and
 value slices into the full [B, H, N, d] tensors; and the driver's order of
 steps, with a recording stand-in for the CUDA shard. The pyramid must see
@@ -55,12 +55,12 @@ def _gather_rank(rank, world, port, shape, errq):
         raise
 
 
-@pytest.mark.parametrize("shape", [(1, 2, 64, 8), (2, 3, 10, 4)])
-def test_gather_sequence_two_ranks(shape):
+@pytest.mark.parametrize("world,shape", [(2, (1, 2, 64, 8)), (2, (2, 3, 10, 4)), (4, (1, 3, 96, 4))])
+def test_gather_sequence_ranks(world, shape):
     ctx = mp.get_context("spawn")
     errq = ctx.SimpleQueue()
     port = _free_port()
-    procs = [ctx.Process(target=_gather_rank, args=(r, 2, port, shape, errq)) for r in range(2)]
+    procs = [ctx.Process(target=_gather_rank, args=(r, world, port, shape, errq)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
