@@ -18,7 +18,10 @@ that suite's items are reproduced. Recipe:
   of that head group's queries at t;
 * ``clustered``: keys are a per-segment mean mu_s ~ N(0, I) (one per
   ``segment`` tokens and kv head) plus 0.5 * N(0, 1); q and v are N(0, 1);
-* ``iid``: q, k, v ~ N(0, 1).
+* ``iid``: q, k, v ~ N(0, 1);
+* ``periodic``: the keys of leaf i repeat those of leaf i mod ``period``
+  (an N(0, 1) pattern of ``period`` leaves per kv head), so blocks of equal
+  content recur and their scores tie exactly; q and v are N(0, 1).
 """
 from __future__ import annotations
 
@@ -42,6 +45,7 @@ class Prefill:
     structure: str = "iid"  # "iid" | "needle" | "clustered"
     n_needles: int = 0
     segment: int = 4096
+    period: int = 3
     seed: int = 0
     g: int = 2
     q_tile: int = 4
@@ -162,6 +166,10 @@ def prefill_inputs(w: Prefill, device="cpu"):
         nseg = (w.N + w.segment - 1) // w.segment
         mu = _randn((w.B, w.H_kv, nseg, w.d), device, w.seed + 3)
         k = 0.5 * k + mu.repeat_interleave(w.segment, dim=2)[:, :, : w.N, :]
+    elif w.structure == "periodic":
+        pat = k[:, :, : w.period * w.C, :]
+        reps = -(-w.N // (w.period * w.C))
+        k = pat.repeat(1, 1, reps, 1)[:, :, : w.N, :].contiguous()
     elif w.structure != "iid":
         raise ValueError(w.structure)
     dt = w.torch_dtype

@@ -175,6 +175,97 @@ def test_inner_level_scores_from_direct_averages(oracle):
     assert n_checked > 20
 
 
+def test_inner_level_causal_scores_leave_out_later_children(oracle):
+    # §TopK inner-level score under the causal reading: a candidate block
+    # whose first key is <= t is usable, but its second child may start after
+    # t; that child's summary must not enter the LSE. The summaries themselves
+    # stay the static whole-block means of §Pyramid (avg_pool1d here), so only
+    # the set of children changes. A filter applied at the leaf level alone
+    # fails this pin.
+    w = _small(N=2048, C=16, K=3, causal=True, H_q=6, H_kv=2, d=16, seed=31)
+    x = workloads.prefill_inputs(w)
+    rng = np.random.default_rng(17)
+    rows = [(0, h, int(t)) for h in range(w.H_kv) for t in rng.integers(4 * w.C, w.N, 120)]
+    _, _, _, _, tr = _trace(oracle, w, x, rows)
+    sizes, _ = oracle.geometry(w.N, w.C)
+    G = w.H_q // w.H_kv
+    k64 = x["k"].double()
+    straddling = 0
+    for r, (b, h, t) in enumerate(rows):
+        q = x["q"][b, h * G:(h + 1) * G, t, :].double()
+        for l in range(2, len(sizes)):
+            n = tr["n"][r, l]
+            if n <= w.K:
+                continue
+            child_span = w.C << (l - 2)
+            child = _dense_pool(k64, child_span)[b, h]  # static level l-1 means
+            for s in range(n):
+                i = tr["cand"][r, l, s]
+                kids = [c for c in (2 * i, 2 * i + 1) if c < sizes[l - 1] and c * child_span <= t]
+                assert kids and kids[0] == 2 * i
+                straddling += len(kids) == 1 and 2 * i + 1 < sizes[l - 1]
+                logits = (q @ child[kids].T) / math.sqrt(w.d)  # [G, |kids|]
+                want = torch.logsumexp(logits, dim=1).sum().item()
+                assert abs(tr["score"][r, l, s] - want) < 1e-9
+    assert straddling > 50
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_ties_break_toward_lower_block_index(oracle, causal):
+    # Tie rule (the pages leave it open; read as: equal scores go to the lower
+    # block index). When every key is the same vector v, every full block of
+    # every level has the same summary v, so all full candidates tie exactly:
+    # a block's LSE over n equal logits is s + log n. A block cut by the causal
+    # limit has fewer usable children and scores strictly lower. Every level
+    # therefore keeps the K lowest full blocks, whose children are again the
+    # lowest, and the selection is exactly leaves 0..K-1 for every query that
+    # can see more than K leaves; the flat and exact selectors agree.
+    w = _small(N=1024, C=16, K=4, causal=causal, H_q=4, H_kv=2, d=16, seed=41)
+    x = workloads.prefill_inputs(w)
+    vec = torch.randn(w.d, generator=torch.Generator().manual_seed(2))
+    k = vec.expand(w.B, w.H_kv, w.N, w.d).contiguous()
+    cfg = _cfg(oracle, w)
+    pyr = oracle.build_pyramid(k, w.C)
+    ts = [t for t in range(0, w.N, 11) if t // w.C + 1 > w.K]
+    rows = [(0, h, t) for h in range(w.H_kv) for t in ts]
+    want = np.tile(np.arange(w.K, dtype=np.int32), (len(rows), 1))
+    sel, gap = oracle.select_rows(cfg, x["q"], k, pyr, rows)
+    assert np.array_equal(sel, want)
+    # The K-th and (K+1)-th candidates tie at some level, except causal rows
+    # whose only scored level holds K full leaves and the cut one.
+    assert (gap >= 0).all() and (gap == 0).mean() > (0.999 if not causal else 0.9)
+    s_flat, _ = oracle.select_flat_rows(cfg, x["q"], pyr, rows)
+    s_exact, _ = oracle.select_exact_rows(cfg, x["q"], k, rows)
+    assert np.array_equal(s_flat, want)
+    assert np.array_equal(s_exact, want)
+
+
+def test_kept_sets_follow_score_then_lower_index_on_recurring_blocks(oracle):
+    # With leaf contents that recur with period 3, blocks of equal content at
+    # every level have identical summaries, so many candidates tie exactly and
+    # the K-th place often falls inside a tied class. At every scored level the
+    # kept set must be the first K candidates when ordered by score (higher
+    # first) and then by block index (lower first).
+    w = _small(N=3000, C=16, K=5, causal=True, H_q=4, H_kv=2, d=16, seed=43, structure="periodic", period=3)
+    x = workloads.prefill_inputs(w)
+    rows = [(0, h, t) for h in range(w.H_kv) for t in range(100, w.N, 13)]
+    _, _, _, _, tr = _trace(oracle, w, x, rows)
+    tied_at_k = 0
+    for r in range(len(rows)):
+        for l in range(1, tr["n"].shape[1]):
+            n = tr["n"][r, l]
+            if n <= w.K:
+                continue
+            cand = tr["cand"][r, l, :n]
+            sc = tr["score"][r, l, :n]
+            order = sorted(range(n), key=lambda m: (-sc[m], cand[m]))
+            want = {int(cand[m]) for m in order[: w.K]}
+            got = {int(c) for c, kk in zip(cand, tr["kept"][r, l, :n]) if kk}
+            assert got == want
+            tied_at_k += sc[order[w.K - 1]] == sc[order[w.K]]
+    assert tied_at_k > 100
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_large_K_selects_everything_and_attention_is_dense(oracle, causal):
     # With K >= number of leaves nothing is ever scored (§TopK keep-all rule),
