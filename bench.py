@@ -152,6 +152,70 @@ def attn_bytes(w) -> float:
     return qo + 2 * w.B * w.H_kv * keys * w.d * e
 
 
+def _valid(w, l, t):
+    """Blocks of level l usable by queries at positions t (numpy array)."""
+    import numpy as np
+    M = -(-w.N // (w.C << (l - 1)))
+    if not w.causal:
+        return np.full(t.shape, M, dtype=np.int64)
+    return np.minimum(M, t // (w.C << (l - 1)) + 1)
+
+
+def work_model(w):
+    """Algorithmic work per launch of each prefill kernel, from the level
+    geometry alone (one pass over every query position t):
+      router: per query row and scored inner level l >= 2, up to 2K
+        candidates, each gathering its <= 2 child summaries (d fp32 values,
+        stored as bf16 hi + lo) from L2;
+      leaf scorer: (query, candidate leaf) pairs at the leaf level, each
+        2 G_Q C d flops;
+      attention: 4 G_Q d flops per usable key of the K selected blocks;
+      flat selector: 2 d flops per (query row, usable leaf) after the group sum;
+      exact selector: 2 G_Q C d flops per (query row, usable leaf)."""
+    import numpy as np
+    t = np.arange(w.N, dtype=np.int64)
+    L = api.pyramid_geometry(w.N, w.C)[0]
+    K, G, e = w.K, w.H_q // w.H_kv, (2 if w.dtype == "bf16" else 4)
+    heads = w.B * w.H_kv
+    gathered = np.zeros(w.N)
+    started = np.zeros(w.N, dtype=bool)
+    for l in range(L, 1, -1):
+        v = _valid(w, l, t)
+        scored = started | (v > K)
+        cand = np.where(started, np.minimum(2 * K, v), v)
+        gathered += np.where(scored, cand * 2, 0)
+        started = scored
+    v1 = _valid(w, 1, t)
+    pairs = np.where(v1 > K, np.where(started, np.minimum(2 * K, v1), v1), 0)
+    keys = np.minimum(K * w.C, t + 1) if w.causal else np.full(w.N, min(K * w.C, w.N))
+    return {k: float(v) for k, v in {
+        "router_gather_bytes": heads * gathered.sum() * w.d * 4,
+        "router_hbm_bytes": w.B * w.H_q * w.N * w.d * e + heads * w.N * (32 + 1) * 4,
+        "leaf_pairs": heads * pairs.sum(),
+        "leaf_flops": heads * pairs.sum() * 2 * G * w.C * w.d,
+        "attn_flops": heads * keys.sum() * 4 * G * w.d,
+        "attn_unique_bytes": (2 * w.B * w.H_q * w.N * w.d * e + 2 * heads * w.N * w.d * e + w.B * w.H_q * w.N * 4),
+        "flat_flops": heads * v1.sum() * 2 * w.d,
+        "exact_flops": heads * v1.sum() * 2 * G * w.C * w.d,
+        "final_bytes": heads * w.N * (32 * 8 + K * 4),
+        "split_bytes": heads * api.pyramid_rows(w.N, w.C) * w.d * 8,
+    }.items()}
+
+
+def decode_bytes(wd) -> float:
+    """HBM bytes one decode step must read, per (sequence, kv head): the
+    group's queries, the child summaries of up to 2K candidates per scored
+    inner level (fp32), the raw keys of up to 2K candidate leaves, and the
+    values of the K selected leaves; plus the append's leaf and ancestor
+    rows. Taken at the workload's starting length."""
+    n = wd.context + 1
+    L = api.pyramid_geometry(n, wd.C)[0]
+    scored_inner = sum(1 for l in range(2, L + 1) if -(-n // (wd.C << (l - 2))) > wd.K)
+    per = (wd.G_Q * wd.d * 2 + scored_inner * 2 * wd.K * 2 * wd.d * 4 + 2 * wd.K * wd.C * wd.d * 2
+           + wd.K * wd.C * wd.d * 2 + L * 3 * wd.d * 4 + 2 * wd.d * 2)
+    return wd.S * wd.H_kv * per
+
+
 def pyramid_bytes(w) -> float:
     e = 2 if w.dtype == "bf16" else 4
     R = api.pyramid_rows(w.N, w.C)
@@ -203,6 +267,58 @@ def measured_traffic(workload: str, kernel: str):
         return rec["dram_read_bytes"] + rec["dram_write_bytes"]
     except (OSError, KeyError, ValueError):
         return None
+
+
+def kernel_rooflines(w, kern, flat_ms, exact_ms, decode, pk, pk_kind):
+    """Each kernel's achieved rate against its binding roof: algorithmic work
+    per launch (work_model, pyramid_bytes, decode_bytes) over the kernel's
+    CUDA-event time per launch. Tensor-bound kernels use the measured bf16
+    dense peak (burst: each is a single launch of at most a few tens of ms);
+    memory-bound ones the measured HBM copy peak."""
+    m = work_model(w)
+    hbm, tf = pk["hbm_gbs"], pk["bf16_tflops"]
+    out = {}
+
+    def add(name, ms, launches, bound, work, note, **extra):
+        if ms is None or ms <= 0:
+            return
+        if bound == "tensor":
+            ach, peak, unit = work / (ms * 1e-3) / 1e12, tf, "TFLOP/s"
+        else:
+            ach, peak, unit = work / (ms * 1e-3) / 1e9, hbm, "GB/s"
+        out[name] = dict(ms=ms, launches=launches, bound=bound, achieved=ach, peak=peak, unit=unit,
+                         frac=ach / peak, peak_kind=pk_kind, work=work,
+                         work_unit="flop" if bound == "tensor" else "byte", note=note, **extra)
+
+    def k(name):
+        return kern.get(name, (None, 0))
+
+    add("pyramid_kernel", *k("pyramid_kernel"), "hbm", pyramid_bytes(w),
+        "keys read once + fp32 pyramid written once (one cooperative launch)")
+    add("split_kernel", *k("split_kernel"), "hbm", m["split_bytes"], "fp32 pyramid read, bf16 hi/lo planes written")
+    r = k("router_kernel")
+    if r[0]:
+        add("router_kernel", *r, "hbm", m["router_hbm_bytes"],
+            "HBM bytes: queries + candidate lists; its real limit is the L2 gather of child summaries",
+            l2_gather_gbs=m["router_gather_bytes"] / (r[0] * 1e-3) / 1e9, l2_gather_bytes=m["router_gather_bytes"])
+    for leaf in ("leaf_umma_kernel", "leaf_kernel"):
+        add(leaf, *k(leaf), "tensor", m["leaf_flops"], f"{m['leaf_pairs']:.4g} (query, leaf) pairs x 2 G_Q C d")
+    add("final_kernel", *k("final_kernel"), "hbm", m["final_bytes"], "2K (score, leaf) pairs read + K written per row")
+    a = k("attn_kernel")
+    if a[0]:
+        add("attn_kernel", *a, "tensor", m["attn_flops"], "4 G_Q d flops per usable key of the K selected blocks",
+            hbm_unique_gbs=m["attn_unique_bytes"] / (a[0] * 1e-3) / 1e9,
+            hbm_unique_frac=m["attn_unique_bytes"] / (a[0] * 1e-3) / 1e9 / hbm,
+            l2_gather_gbs=attn_bytes(w) / (a[0] * 1e-3) / 1e9)
+    add("flat_mma_kernel", flat_ms, 1, "tensor", m["flat_flops"],
+        "2 d flops per (query row, usable leaf) after the group sum; not part of the step")
+    add("exact_umma_kernel", exact_ms, 1, "tensor", m["exact_flops"],
+        "2 G_Q C d flops per (query row, usable leaf); not part of the step")
+    if decode:
+        wd = workloads.DECODE[decode["workload"]]
+        add("decode_kernel", decode["us_per_step"] * 1e-3, 1, "hbm", decode_bytes(wd),
+            "fused step: summaries of scored levels, candidate leaf keys, selected values, append rows")
+    return out
 
 
 # ------------------------------------------------------------------ arms
@@ -299,44 +415,64 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.B * w.N / v * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "C": w.C,
-                       "K": w.K, "causal": w.causal, "input_dtype": w.dtype},
+                       "g": 2, "K": w.K, "q_tile": 4, "causal": w.causal, "structure": w.structure,
+                       "input_dtype": w.dtype},
+            "ms_per_step_kind": "extrapolated: each step times the full pyramid plus a random row sample and "
+                                "scales the row time linearly to all rows",
             "cpu_baseline": dict(vals[-1], value=v),
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
 
 
-def time_decode(wd, steps=32, warmup=4):
-    """µs per decode step (append + fused select + attention) on the decode workload."""
+def _reset_decode(st, lens0):
+    """Back to the cached context: lengths restored, pyramids rebuilt."""
+    st.len.copy_(lens0)
+    st.init()
+
+
+def time_decode(wd, warmup=4):
+    """µs per decode step over the workload's full run of wd.steps steps
+    (context -> context + steps tokens per sequence): append + fused select
+    + attention per step. Then, from the same starting state, the selection
+    alone, the attention alone and the append alone, each over wd.steps
+    launches. Warm-up steps run first and the state is reset after them."""
     dev = torch.device("cuda")
+    steps = wd.steps
     kc, vc, lens = workloads.decode_cache(wd, device=dev)
+    lens0 = lens.clone()
     st = api.DecodeState(S=wd.S, cap=wd.cap, H_q=wd.H_q, H_kv=wd.H_kv, d=wd.d, C=wd.C, K=wd.K,
                          dtype=wd.torch_dtype, device=dev, k_cache=kc, v_cache=vc, lens=lens)
     st.init()
-    ins = [workloads.decode_step_inputs(wd, s, device=dev) for s in range(steps + warmup)]
+    ins = [workloads.decode_step_inputs(wd, s, device=dev) for s in range(steps)]
     for s in range(warmup):
         st.step(*ins[s], keep_sel=False)
+    _reset_decode(st, lens0)
     e0, e1 = events(2)
     torch.cuda.synchronize()
     e0.record()
-    for s in range(warmup, warmup + steps):
+    for s in range(steps):
         st.step(*ins[s], keep_sel=False)
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / steps
-    # Selection alone on the same state.
+    ok = int(st.status.item()) == 0
+    end_len = int(st.len.min().item())
+    _reset_decode(st, lens0)
     q = ins[0][0]
+    st.select(q)
+    torch.cuda.synchronize()
     e0.record()
-    for _ in range(steps):
-        st.select(q)
+    for s in range(steps):
+        st.select(ins[s][0])
     e1.record()
     torch.cuda.synchronize()
     us_sel = e0.elapsed_time(e1) * 1e3 / steps
     # Attention alone over the selection just made, then the append alone
     # (each its own launch; the append advances every sequence by one token).
     e0.record()
-    for _ in range(steps):
-        st.attend(q)
+    for s in range(steps):
+        st.attend(ins[s][0])
     e1.record()
     torch.cuda.synchronize()
     us_attn = e0.elapsed_time(e1) * 1e3 / steps
@@ -346,17 +482,19 @@ def time_decode(wd, steps=32, warmup=4):
     e1.record()
     torch.cuda.synchronize()
     us_app = e0.elapsed_time(e1) * 1e3 / steps
-    ok = int(st.status.item()) == 0
+    ok = ok and int(st.status.item()) == 0
     del st, kc, vc
     torch.cuda.empty_cache()
     return {"workload": wd.name, "us_per_step": us, "select_us": us_sel, "attn_us": us_attn, "append_us": us_app,
-            "steps": steps, "status_ok": ok}
+            "steps": steps, "tokens": [wd.context, end_len], "status_ok": ok}
 
 
-def time_decode_paged(wd, steps=32, warmup=4):
-    """µs per fused decode step over paged caches: the same workload with each
-    sequence's leaf blocks in pages of a shuffled pool (one leaf per page)."""
+def time_decode_paged(wd, warmup=4):
+    """µs per fused decode step over paged caches: the same workload and
+    number of steps with each sequence's leaf blocks in pages of a shuffled
+    pool (one leaf per page)."""
     dev = torch.device("cuda")
+    steps = wd.steps
     kc, vc, lens = workloads.decode_cache(wd, device=dev)
     max_pages = wd.cap // wd.C
     perm = torch.randperm(wd.S * max_pages, generator=torch.Generator().manual_seed(1)).to(dev)
@@ -372,16 +510,18 @@ def time_decode_paged(wd, steps=32, warmup=4):
     vp = pages(vc)
     del vc
     bt = perm.reshape(wd.S, max_pages).to(torch.int32).contiguous()
+    lens0 = lens.clone()
     st = api.PagedDecodeState(S=wd.S, max_pages=max_pages, H_q=wd.H_q, H_kv=wd.H_kv, d=wd.d, C=wd.C, K=wd.K,
                               k_pages=kp, v_pages=vp, block_table=bt, lens=lens, dtype=wd.torch_dtype)
     st.init()
-    ins = [workloads.decode_step_inputs(wd, s, device=dev) for s in range(steps + warmup)]
+    ins = [workloads.decode_step_inputs(wd, s, device=dev) for s in range(steps)]
     for s in range(warmup):
         st.step(*ins[s], keep_sel=False)
+    _reset_decode(st, lens0)
     e0, e1 = events(2)
     torch.cuda.synchronize()
     e0.record()
-    for s in range(warmup, warmup + steps):
+    for s in range(steps):
         st.step(*ins[s], keep_sel=False)
     e1.record()
     torch.cuda.synchronize()
@@ -438,6 +578,13 @@ def run_gpu(args):
     dev_ms = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
     ms, value = aggregate(dist, dev_ms, w.B * w.N)
     stage_ms = {kk: vv / args.steps for kk, vv in stage.items()}
+
+    # Per-kernel device time: the same steps again, outside the timed region,
+    # with every library launch bracketed by CUDA events on its stream.
+    with api.KernelTimer() as kt:
+        for _ in range(args.steps):
+            p(q, k, v)
+    kern_ms = {n: (t_ms / args.steps, c / args.steps) for n, (t_ms, c) in kt.result.items()}
 
     # Exact-score flat selector (every usable leaf scored by its raw-key LSE)
     # on the same inputs, once after a warm-up, and the share of its top-K
@@ -555,16 +702,18 @@ def run_gpu(args):
             decode["cpu_baseline"] = cpu_decode_baseline(workloads.DECODE[args.decode_workload])
 
     pk, pk_kind = peaks()
-    # Roofline of the dominant stage (the attention kernel: one launch per step).
-    a_bytes = attn_bytes(w)
-    a_ms = stage_ms["attn"]
-    roof = {"kernel": "attn_kernel (pisa_sparse_attn_fwd)", "bound": "hbm",
-            "achieved": a_bytes / (a_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "peak_kind": pk_kind, "traffic": measured_traffic(w.name, "attn"), "algorithmic_bytes": a_bytes,
-            "note": "algorithmic bytes = q + out once plus the K/V rows of each row's K causally clipped "
-                    "blocks (no cross-query reuse); most of them are served from L2, so frac > 1 of the "
-                    "HBM copy peak is possible; traffic = measured DRAM bytes per launch"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    kernels = kernel_rooflines(w, kern_ms, flat_ms, exact_ms, decode, pk, pk_kind)
+    # Roofline of the dominant kernel of the step (largest share of its time).
+    step_kernels = [n for n in kern_ms if n in kernels]
+    top = max(step_kernels, key=lambda n: kernels[n]["ms"])
+    kr = kernels[top]
+    roof = {"kernel": top, "bound": kr["bound"], "achieved": kr["achieved"], "peak": kr["peak"], "unit": kr["unit"],
+            "frac": kr["frac"], "peak_kind": pk_kind, "share_of_step": kr["ms"] / ms,
+            "traffic": measured_traffic(w.name, top), "work_per_launch": kr["work"], "work_unit": kr["work_unit"],
+            "note": kr["note"]}
+    for extra in ("hbm_unique_frac", "l2_gather_gbs"):
+        if extra in kr:
+            roof[extra] = kr[extra]
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -573,7 +722,7 @@ def run_gpu(args):
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "C": w.C,
                    "g": 2, "K": w.K, "q_tile": 4, "causal": w.causal, "structure": w.structure,
                    "l2": "inputs larger than L2 (q alone is %.0f MB)" % (q.numel() * q.element_size() / 1e6)},
-        "stages_ms": stage_ms, "flat_select_ms": flat_ms,
+        "stages_ms": stage_ms, "kernels": kernels, "flat_select_ms": flat_ms,
         "select_speedup_vs_flat": flat_ms / stage_ms["select"] if stage_ms["select"] > 0 else None,
         "exact_select_ms": exact_ms,
         "select_speedup_vs_exact": exact_ms / stage_ms["select"] if stage_ms["select"] > 0 else None,

@@ -52,12 +52,16 @@ SIGNATURES = {
     "pisa_version": (_i32, []),
     "pisa_launch_count": (ctypes.c_uint64, []),
     "pisa_device_faults": (ctypes.c_uint64, []),
+    "pisa_timing_start": (_i32, []),
+    "pisa_timing_stop": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                        ctypes.POINTER(ctypes.c_int)]),
     "pisa_pyramid_geometry": (_i32, [_i64, _i32, _i32, ctypes.POINTER(_i32), _p]),
     "pisa_pyramid_rows": (_i64, [_i64, _i32]),
     "pisa_build_pyramid": (_i32, [_PC, _p, _p, _p]),
     "pisa_select_workspace_bytes": (ctypes.c_size_t, [_PC]),
     "pisa_select": (_i32, [_PC, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
-    "pisa_select_flat": (_i32, [_PC, _p, _p, _p, _p]),
+    "pisa_select_flat_workspace_bytes": (ctypes.c_size_t, [_PC]),
+    "pisa_select_flat": (_i32, [_PC, _p, _p, _p, _p, ctypes.c_size_t, _p]),
     "pisa_select_exact": (_i32, [_PC, _p, _p, _p, _p]),
     "pisa_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_PC]),
     "pisa_sparse_attn_bwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),

@@ -43,6 +43,18 @@ def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
 def _on_cuda(t: torch.Tensor, name: str):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    _check_device_index(t.device.index, name)
+
+
+def _check_device_index(index, name: str):
+    """The C library launches on the runtime's current device, so every tensor
+    of a call must live there: another GPU's pointers would reach the kernels
+    and their TMA descriptors. Make the tensors' device current first
+    (torch.cuda.set_device or a torch.cuda.device(...) block)."""
+    cur = torch.cuda.current_device()
+    if index is not None and index != cur:
+        raise ValueError(f"{name} is on cuda:{index} but the current device is cuda:{cur}; "
+                         f"call under torch.cuda.device({index})")
 
 
 def launch_count() -> int:
@@ -53,6 +65,30 @@ def launch_count() -> int:
 def device_faults() -> int:
     """Bounded device waits that ran out of time on the current device (synchronises)."""
     return int(_lib.lib().pisa_device_faults())
+
+
+class KernelTimer:
+    """Per-kernel device time of every library launch inside a ``with`` block
+    (pisa_timing_start / pisa_timing_stop): CUDA events on each launching
+    stream. On exit, ``result`` maps kernel name -> (total ms, launches).
+    Exiting synchronises with the timed streams."""
+
+    MAX = 64
+
+    def __enter__(self):
+        _lib.call("pisa_timing_start")
+        self.result = {}
+        return self
+
+    def __exit__(self, *exc):
+        names = (ctypes.c_char_p * self.MAX)()
+        ms = (ctypes.c_double * self.MAX)()
+        cnt = (ctypes.c_int * self.MAX)()
+        n = _lib.lib().pisa_timing_stop(self.MAX, names, ms, cnt)
+        if n < 0:
+            raise RuntimeError("pisa_timing_stop: a timing event failed")
+        self.result = {names[i].decode(): (ms[i], cnt[i]) for i in range(min(n, self.MAX))}
+        return False
 
 
 def pyramid_geometry(N: int, C: int, g: int = 2):
@@ -140,7 +176,8 @@ def select(q, k, pyr, *, C: int, K: int, causal: bool, scale: float = 0.0, out=N
     return out
 
 
-def select_flat(q, pyr, *, C: int, K: int, causal: bool, H_kv: int, scale: float = 0.0, out=None):
+def select_flat(q, pyr, *, C: int, K: int, causal: bool, H_kv: int, scale: float = 0.0, out=None,
+                workspace=None):
     """Flat single-level top-K over all leaf summaries: sel [B, H_kv, N, K] int32."""
     _need(q, "q")
     B, H_q, N, d = q.shape
@@ -149,7 +186,12 @@ def select_flat(q, pyr, *, C: int, K: int, causal: bool, H_kv: int, scale: float
     if out is None:
         out = torch.empty((B, H_kv, N, K), dtype=torch.int32, device=q.device)
     _need(out, "out", torch.int32, (B, H_kv, N, K))
-    _lib.call("pisa_select_flat", ctypes.byref(pr.cstruct()), _p(q), _p(pyr), _p(out), _stream(q))
+    need = int(_lib.lib().pisa_select_flat_workspace_bytes(ctypes.byref(pr.cstruct())))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
+    _lib.call("pisa_select_flat", ctypes.byref(pr.cstruct()), _p(q), _p(pyr), _p(out), _p(workspace),
+              workspace.numel() * workspace.element_size(), _stream(q))
     return out
 
 

@@ -175,13 +175,25 @@ pisa_status pisa_select(const pisa_config* cfg, const void* q, const void* k, co
   return pisa_select_span(cfg, &all, q, k, pyr, sel, sel_score, ws, ws_bytes, stream);
 }
 
-pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float* pyr, int32_t* sel, void* stream) {
+size_t pisa_select_flat_workspace_bytes(const pisa_config* cfg) {
+  if (check_cfg(cfg) != PISA_OK) return 0;
+  return flat_umma_workspace_bytes(args_of(cfg));
+}
+
+pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float* pyr, int32_t* sel, void* ws,
+                             size_t ws_bytes, void* stream) {
   pisa_status s = check_cfg(cfg);
   if (s != PISA_OK) return s;
   if (!q || !pyr || !sel || !aligned16(q) || !aligned16(pyr) || !aligned16(sel)) return PISA_ERR_INVALID_ARGUMENT;
   const Layout lay = make_layout(cfg->N, cfg->C);
-  if (cfg->dtype == PISA_DTYPE_BF16) return from_cuda(launch_flat_mma(args_of(cfg), q, pyr, lay.R, sel, as_stream(stream)));
-  return from_cuda(launch_flat_rows(args_of(cfg), q, pyr, lay.R, sel, as_stream(stream)));
+  const PrefillArgs a = args_of(cfg);
+  if (flat_umma_supported(a)) {
+    const size_t need = flat_umma_workspace_bytes(a);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return PISA_ERR_WORKSPACE;
+    return from_cuda(launch_flat_umma(a, q, pyr, lay.R, sel, ws, as_stream(stream)));
+  }
+  if (cfg->dtype == PISA_DTYPE_BF16) return from_cuda(launch_flat_mma(a, q, pyr, lay.R, sel, as_stream(stream)));
+  return from_cuda(launch_flat_rows(a, q, pyr, lay.R, sel, as_stream(stream)));
 }
 
 pisa_status pisa_select_exact(const pisa_config* cfg, const void* q, const void* k, int32_t* sel, void* stream) {

@@ -308,6 +308,7 @@ cudaError_t launch_attn_mma(const PrefillArgs& a, const void* q, const void* k, 
     auto kern = a.C == 64 ? attn_kernel<D, 64, G> : attn_kernel<D, 32, G>;
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e2 != cudaSuccess) return e2;
+    TimedLaunch tl("attn_kernel", st);
     kern<<<grid, kAttnWarps * 32, smem, st>>>(static_cast<const bf16*>(q), tmk, tmv, sel, a, static_cast<bf16*>(out),
                                               lse, faults);
     count_launch();

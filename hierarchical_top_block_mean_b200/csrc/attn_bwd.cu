@@ -619,19 +619,32 @@ cudaError_t launch_attn_bwd(const PrefillArgs& a, const void* q, const void* k, 
   const unsigned eg = static_cast<unsigned>(eblocks < 148 * 64 ? eblocks : 148 * 64);
   e = dispatch_td(PISA_DTYPE_BF16, a.d, [&](auto, auto dd) -> cudaError_t {
     constexpr int D = decltype(dd)::value;
+    TimedLaunch tl("bwd_prep_kernel", st);
     bwd_prep_kernel<D><<<static_cast<unsigned>((qrows * 32 + 255) / 256), 256, 0, st>>>(
         static_cast<const bf16*>(dout), static_cast<const bf16*>(out), w.D, qrows);
     count_launch();
     return cudaGetLastError();
   });
   if (e != cudaSuccess) return e;
-  bwd_count_kernel<<<eg, 256, 0, st>>>(sel, entries, a.K, a.N, M1, w.count);
+  {
+    TimedLaunch tl("bwd_count_kernel", st);
+    bwd_count_kernel<<<eg, 256, 0, st>>>(sel, entries, a.K, a.N, M1, w.count);
+  }
   count_launch();
-  bwd_scan_kernel<<<1, 1024, 0, st>>>(w.count, nb, w.off, w.item_off);
+  {
+    TimedLaunch tl("bwd_scan_kernel", st);
+    bwd_scan_kernel<<<1, 1024, 0, st>>>(w.count, nb, w.off, w.item_off);
+  }
   count_launch();
-  bwd_scatter_kernel<<<eg, 256, 0, st>>>(sel, entries, a.K, a.N, M1, w.off, w.fill, w.qlist);
+  {
+    TimedLaunch tl("bwd_scatter_kernel", st);
+    bwd_scatter_kernel<<<eg, 256, 0, st>>>(sel, entries, a.K, a.N, M1, w.off, w.fill, w.qlist);
+  }
   count_launch();
-  bwd_itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(w.off, w.item_off, nb, M1, w.items);
+  {
+    TimedLaunch tl("bwd_itemize_kernel", st);
+    bwd_itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(w.off, w.item_off, nb, M1, w.items);
+  }
   count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -647,8 +660,11 @@ cudaError_t launch_attn_bwd(const PrefillArgs& a, const void* q, const void* k, 
     auto kq = a.C == 64 ? bwd_dq_kernel<D, 64, GG> : bwd_dq_kernel<D, 32, GG>;
     cudaError_t e2 = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_dq));
     if (e2 != cudaSuccess) return e2;
-    kq<<<grid, kDqWarps * 32, smem_dq, st>>>(static_cast<const bf16*>(q), tmk, tmv, sel,
-                                            static_cast<const bf16*>(dout), lse, w.D, a, dq, faults);
+    {
+      TimedLaunch tl("bwd_dq_kernel", st);
+      kq<<<grid, kDqWarps * 32, smem_dq, st>>>(static_cast<const bf16*>(q), tmk, tmv, sel,
+                                              static_cast<const bf16*>(dout), lse, w.D, a, dq, faults);
+    }
     count_launch();
     if ((e2 = cudaGetLastError()) != cudaSuccess) return e2;
     const int smem_kv = a.C == 64 ? DkvSmem<D, 64, GG>::kBytes : DkvSmem<D, 32, GG>::kBytes;
@@ -658,6 +674,7 @@ cudaError_t launch_attn_bwd(const PrefillArgs& a, const void* q, const void* k, 
     int per_sm = 0;
     e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kk, kDkvWarps * 32, smem_kv);
     if (e2 != cudaSuccess) return e2;
+    TimedLaunch tl("bwd_dkdv_kernel", st);
     kk<<<static_cast<unsigned>(sm_count_bwd() * (per_sm > 0 ? per_sm : 1)), kDkvWarps * 32, smem_kv, st>>>(
         static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
         static_cast<const bf16*>(dout), lse, w.D, w.items, w.item_off + nb, w.qlist, a, dk, dv);

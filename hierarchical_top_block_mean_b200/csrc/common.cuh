@@ -22,6 +22,23 @@ using bf16 = __nv_bfloat16;
 // ------------------------------------------------------------ host counter
 void count_launch(int n = 1);
 
+// ---------------------------------------------------- per-kernel timing
+// Between pisa_timing_start() and pisa_timing_stop() every launch site
+// brackets its kernel with two CUDA events recorded on the launching stream:
+// a TimedLaunch is constructed just before the launch and destroyed just
+// after it. Outside that window construction and destruction do nothing.
+class TimedLaunch {
+ public:
+  TimedLaunch(const char* name, cudaStream_t st);
+  ~TimedLaunch();
+  TimedLaunch(const TimedLaunch&) = delete;
+  TimedLaunch& operator=(const TimedLaunch&) = delete;
+
+ private:
+  int slot_;
+  cudaStream_t st_;
+};
+
 // ----------------------------------------------------------------- geometry
 // Pyramid level sizes (paper §Pyramid): M_1 = ceil(n / C), M_{l+1} =
 // ceil(M_l / 2). Because ceil(ceil(x / a) / b) = ceil(x / (a b)) for positive

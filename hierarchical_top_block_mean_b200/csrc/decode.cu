@@ -125,6 +125,7 @@ cudaError_t launch_decode_append(const DecodeArgs& a, const Layout& lay, const v
     using T = typename decltype(tt)::type;
     constexpr int D = decltype(dd)::value;
     const int threads = 32 * (a.H_kv < 8 ? a.H_kv : 8);
+    TimedLaunch tl("decode_append_kernel", st);
     decode_append_kernel<T, D><<<a.S, threads, 0, st>>>(a, lay, static_cast<const T*>(k_new),
                                                          static_cast<const T*>(v_new), static_cast<T*>(k_cache),
                                                          static_cast<T*>(v_cache), pyr, len, status);
@@ -140,6 +141,7 @@ cudaError_t launch_decode_rows(const DecodeArgs& a, const Layout& lay, int mode,
     using T = typename decltype(tt)::type;
     constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
     const unsigned blocks = static_cast<unsigned>((static_cast<int64_t>(a.S) * a.H_kv + kRowWarps - 1) / kRowWarps);
+    TimedLaunch tl("decode_rows_kernel", st);
     decode_rows_kernel<T, D, G><<<blocks, kRowWarps * 32, 0, st>>>(
         a, lay, mode, static_cast<const T*>(q_new), static_cast<const T*>(k_cache), static_cast<const T*>(v_cache),
         pyr, len, sel, static_cast<T*>(out), lse);

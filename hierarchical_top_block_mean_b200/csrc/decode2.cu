@@ -608,6 +608,7 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, const Layout& lay, int mode
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    TimedLaunch tl("decode_kernel", st);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, lay, mode, static_cast<const bf16*>(q_new),
                                        static_cast<const bf16*>(k_new), static_cast<const bf16*>(v_new),
                                        static_cast<bf16*>(k_cache), static_cast<bf16*>(v_cache), pyr, len, sel,

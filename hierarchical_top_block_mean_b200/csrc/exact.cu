@@ -271,6 +271,7 @@ cudaError_t launch_exact_umma(const PrefillArgs& a, const void* q, const void* k
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e2 != cudaSuccess) return e2;
     dim3 grid(static_cast<unsigned>((a.N + kQT - 1) / kQT), static_cast<unsigned>(a.B * a.H_kv));
+    TimedLaunch tl("exact_umma_kernel", st);
     kern<<<grid, kExThreads, smem, st>>>(static_cast<const bf16*>(q), tmk, a, sel, wait_fault_counter());
     count_launch();
     return cudaGetLastError();

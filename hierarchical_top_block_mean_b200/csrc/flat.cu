@@ -215,6 +215,7 @@ cudaError_t launch_flat_mma(const PrefillArgs& a, const void* q, const float* py
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     dim3 grid(static_cast<unsigned>((a.N + kFlatRows - 1) / kFlatRows), a.B * a.H_kv);
+    TimedLaunch tl("flat_mma_kernel", st);
     kern<<<grid, kFlatWarps * 32, smem, st>>>(static_cast<const bf16*>(q), pyr, R, a, sel);
     count_launch();
     return cudaGetLastError();

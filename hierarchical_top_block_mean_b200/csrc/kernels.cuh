@@ -37,6 +37,11 @@ cudaError_t launch_attn_mma(const PrefillArgs& a, const void* q, const void* k, 
 
 cudaError_t launch_flat_mma(const PrefillArgs& a, const void* q, const float* pyr, int64_t R, int32_t* sel,
                             cudaStream_t st);
+// tcgen05 flat selection (bf16, d = 128) with its hi/lo operand planes in ws.
+bool flat_umma_supported(const PrefillArgs& a);
+size_t flat_umma_workspace_bytes(const PrefillArgs& a);
+cudaError_t launch_flat_umma(const PrefillArgs& a, const void* q, const float* pyr, int64_t R, int32_t* sel, void* ws,
+                             cudaStream_t st);
 
 // ---- decode
 cudaError_t launch_decode_append(const DecodeArgs& a, const Layout& lay, const void* k_new, const void* v_new,

@@ -16,12 +16,12 @@
 //     rows, N = 64 keys, K = 16 each) into a ring of TMEM accumulators,
 //     then tcgen05.commit to release the query stage (and, after an item's
 //     last tile, the key tile) and to publish the accumulator;
-//   warps 0-7 (epilogue): warps w and w + 4 share TMEM lane quarter w; each
-//     thread owns one lane = one (query, head) row and loads 32 of its 64 key
-//     scores with tcgen05.ld; each half takes a partial max and exp-sum over
-//     its usable keys, the halves are combined through shared memory into the
-//     row's LSE, the 8 heads of a query are summed with three shuffles, and
-//     one lane per query stores the leaf score.
+//   warps 0-7 (epilogue): two groups of four warps take alternate tiles;
+//     warp w reads TMEM lane quarter w & 3, each thread owns one lane = one
+//     (query, head) row and loads its 64 key scores with tcgen05.ld, takes the
+//     max and exp-sum over its usable keys into the row's LSE, the 8 heads of
+//     a query are summed with three shuffles, and one lane per query stores
+//     the leaf score.
 // Operands sit in shared memory as 128-byte-swizzled K-major tiles (rows of
 // 64 bf16, 8-row groups 1 KB apart), which is both the bulk-copy layout and
 // the MMA descriptor layout. Every mbarrier wait is bounded in time; the
@@ -35,9 +35,8 @@ namespace pisa {
 
 namespace {
 
-constexpr int kEpiSplit = 2;               // epilogue warps per TMEM lane quarter (split of the 64 columns)
-constexpr int kEpiWarps = 4 * kEpiSplit;   // warps 0 .. kEpiWarps - 1
-constexpr int kEpiCols = 64 / kEpiSplit;   // key columns per epilogue warp
+constexpr int kEpiGroups = 2;              // epilogue warp groups, taking alternate tiles
+constexpr int kEpiWarps = 4 * kEpiGroups;  // warps 0 .. kEpiWarps - 1
 constexpr int kLoadWarps = 4;              // warps 8-11 gather the query rows
 constexpr int kMmaWarp = kEpiWarps + kLoadWarps;  // warp 12 issues the MMAs
 constexpr int kUmmaThreads = 32 * (kMmaWarp + 1);
@@ -61,7 +60,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ uint64_t kfull[2], kempty[2], qfull[kQStages], qempty[kQStages], accfull[kAccStages], accempty[kAccStages];
   __shared__ uint32_t tmem_base_sh;
-  __shared__ float2 xch[2][kEpiSplit - 1][4][32];  // per tile parity, part >= 1 and quarter: (max, sum) per row
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* kbuf = smem;                       // [2][kKeyBytes]
@@ -74,7 +72,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     }
     for (int i = 0; i < kAccStages; ++i) {
       mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], kEpiWarps);
+      mbar_init(&accempty[i], 4);  // the four warps of the group that owns the tile
     }
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&qfull[i], kLoaders);
@@ -213,105 +211,78 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    // Tiles are walked as one stream; each row's (query, slot) word is
-    // loaded one tile ahead so its latency hides behind the current tile.
+    // Warps 0-3 take the even tiles of the stream and warps 4-7 the odd
+    // ones, so the two groups overlap one tile's TMEM load and barrier waits
+    // with the other's exponentials. Warp w of a group reads TMEM lane
+    // quarter w & 3; each thread owns one (query, head) row and all 64 of
+    // its key scores.
     const float sl2 = a.scale * 1.4426950408889634f;
-    const int qtr = warp & 3, hf = warp >> 2;  // TMEM lane quarter; part of the 64 key columns
-    const int row = 32 * qtr + lane;            // TMEM lane = (query, head) row of the tile
+    const int qtr = warp & 3, grp = warp >> 2;
+    const int row = 32 * qtr + lane;  // TMEM lane = (query, head) row of the tile
     int na = 0;
     int item = blockIdx.x;
     Cursor2 c = cursor(item, info(item));
     int4 inf_next = info(item + gridDim.x);
     int tl = 0;
-    auto pair_word = [&](const Cursor2& cc, int t) -> uint32_t {
-      const int p = cc.p_lo + t * kTilePairs + row / 8;
-      return p < cc.p_hi ? ws.pairs[p] : 0xffffffffu;
-    };
-    uint32_t w_next = item < total ? pair_word(c, 0) : 0xffffffffu;
     while (item < total) {
-      const uint32_t w = w_next;
-      const bool ok = w != 0xffffffffu;
-      const int64_t bh = c.bh;
-      const int64_t key0 = static_cast<int64_t>(c.leaf) * 64;
-      const int nkeys = static_cast<int>(min(static_cast<int64_t>(64), a.N - key0));
-      // Advance the stream and prefetch the next tile's word.
-      Cursor2 cn = c;
-      int tln = tl + 1, itemn = item;
-      if (tln >= c.ntiles) {
-        itemn = item + gridDim.x;
-        tln = 0;
-        if (itemn < total) {
-          cn = cursor(itemn, inf_next);
-          inf_next = info(itemn + gridDim.x);
+      if ((na & 1) == grp) {
+        const int p = c.p_lo + tl * kTilePairs + row / 8;
+        const uint32_t w = p < c.p_hi ? ws.pairs[p] : 0xffffffffu;
+        const bool ok = w != 0xffffffffu;
+        const int64_t key0 = static_cast<int64_t>(c.leaf) * 64;
+        int nv = static_cast<int>(min(static_cast<int64_t>(64), a.N - key0));
+        if (causal && ok)  // the pair holds the query's row; its position is q0 + row
+          nv = static_cast<int>(min(static_cast<int64_t>(nv), a.q0 + static_cast<int64_t>(w >> 5) - key0 + 1));
+        const int as = na % kAccStages;
+        mbar_wait(&accfull[as], (na / kAccStages) & 1, faults);
+        __syncwarp();  // the TMEM load below is warp-collective
+        tc_fence_after();
+        uint32_t v[kAccCols];
+        tmem_ld_cols<kAccCols>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + as * kAccCols, v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty[as]);
+        // Max and sum of exponentials over the usable keys (four chains each).
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (nv >= kAccCols) {
+#pragma unroll
+          for (int j = 0; j < kAccCols; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < kAccCols; ++j)
+            if (j < nv) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
         }
-      }
-      w_next = itemn < total ? pair_word(cn, tln) : 0xffffffffu;
-
-      const int as = na % kAccStages;
-      const int xb = na & 1;
-      mbar_wait(&accfull[as], (na / kAccStages) & 1, faults);
-      __syncwarp();  // the TMEM load below is warp-collective
-      tc_fence_after();
-      uint32_t v[kEpiCols];
-      tmem_ld_cols<kEpiCols>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + as * kAccCols + kEpiCols * hf, v);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[as]);
-      ++na;
-      int nv = nkeys;
-      if (causal && ok)  // the pair holds the query's row; its position is q0 + row
-        nv = static_cast<int>(min(static_cast<int64_t>(nv), a.q0 + static_cast<int64_t>(w >> 5) - key0 + 1));
-      // This warp's columns [kEpiCols hf, kEpiCols (hf + 1)): partial max and
-      // sum of exp (four chains each), then the parts of a row are combined.
-      const int nvh = nv - kEpiCols * hf;
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (nvh >= kEpiCols) {
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        const float mxs = mx * sl2;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (nv >= kAccCols) {
 #pragma unroll
-        for (int j = 0; j < kEpiCols; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
-      } else {
+          for (int j = 0; j < kAccCols; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+        } else {
 #pragma unroll
-        for (int j = 0; j < kEpiCols; ++j)
-          if (j < nvh) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(v[j]));
-      }
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      const float mxs = mx * sl2;
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (nvh >= kEpiCols) {
-#pragma unroll
-        for (int j = 0; j < kEpiCols; ++j) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
-      } else {
-#pragma unroll
-        for (int j = 0; j < kEpiCols; ++j)
-          if (j < nvh) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
-      }
-      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      if (hf > 0) xch[xb][hf - 1][qtr][lane] = make_float2(mx, sum);
-      named_sync(1 + qtr, 32 * kEpiSplit);  // the epilogue warps of this lane quarter
-      if (hf == 0) {
-        float2 part[kEpiSplit];
-        part[0] = make_float2(mx, sum);
-#pragma unroll
-        for (int i = 1; i < kEpiSplit; ++i) part[i] = xch[xb][i - 1][qtr][lane];
-        float m = part[0].x;
-#pragma unroll
-        for (int i = 1; i < kEpiSplit; ++i) m = fmaxf(m, part[i].x);
-        float z = 0.f;
-#pragma unroll
-        for (int i = 0; i < kEpiSplit; ++i)
-          if (part[i].x != -INFINITY) z += part[i].y * ex2_approx((part[i].x - m) * sl2);
-        float u = ok ? m * a.scale + logf(z) : 0.f;
+          for (int j = 0; j < kAccCols; ++j)
+            if (j < nv) s4[j & 3] += ex2_approx(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+        }
+        const float z = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        float u = ok && nv > 0 ? mx * a.scale + logf(z) : 0.f;
         u += __shfl_xor_sync(kFull, u, 1);
         u += __shfl_xor_sync(kFull, u, 2);
         u += __shfl_xor_sync(kFull, u, 4);
         if (ok && (row & 7) == 0) {
-          const int64_t orow = bh * a.Nq + static_cast<int64_t>(w >> 5);
+          const int64_t orow = static_cast<int64_t>(c.bh) * a.Nq + static_cast<int64_t>(w >> 5);
           ws.score[orow * 32 + (w & 31)] = u;
         }
       }
-      c = cn;
-      tl = tln;
-      item = itemn;
+      ++na;
+      if (++tl >= c.ntiles) {
+        item += gridDim.x;
+        tl = 0;
+        if (item < total) {
+          c = cursor(item, inf_next);
+          inf_next = info(item + gridDim.x);
+        }
+      }
     }
   }
   tc_fence_before();
@@ -347,6 +318,7 @@ cudaError_t launch_leaf_umma(const PrefillArgs& a, const void* q, const void* k,
   const size_t smem = 2 * static_cast<size_t>(kKeyBytes) + kQStages * static_cast<size_t>(kQStageBytes) + 1024;
   e = cudaFuncSetAttribute(leaf_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  TimedLaunch tl("leaf_umma_kernel", st);
   leaf_umma_kernel<<<static_cast<unsigned>(sm_count_umma()), kUmmaThreads, smem, st>>>(
       static_cast<const bf16*>(q), tmk, a, ws, nb, M1, wait_fault_counter());
   count_launch();

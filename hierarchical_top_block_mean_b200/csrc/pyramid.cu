@@ -6,9 +6,15 @@
 // in fp32; each pyramid row is written once. The leaf pass also builds the
 // first kSubLevels levels above the leaves inside the CTA (from shared
 // memory); upper passes then fold 2^kUpperLevels nodes per CTA until the
-// root. All passes use the same two-child mean so that every route to a row
-// (batch build, decode init, decode append) produces identical bits.
+// root. One cooperative launch runs every pass, with grid-wide barriers
+// between them, so a small pyramid costs one launch, not one per pass. All
+// passes use the same two-child mean so that every route to a row (batch
+// build, decode init, decode append) produces identical bits.
+#include <cooperative_groups.h>
+
 #include "pyramid.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace pisa {
 
@@ -18,6 +24,7 @@ constexpr int kLeafWarps = 8;    // leaves per CTA in the leaf pass (one per war
 constexpr int kSubLevels = 3;    // log2(kLeafWarps): levels 2..4 built in-CTA
 constexpr int kUpperNodes = 32;  // input nodes per CTA in an upper pass
 constexpr int kUpperLevels = 5;  // log2(kUpperNodes)
+constexpr int kThreads = kLeafWarps * 32;
 
 // Tokens of sequence b: len[b] when given (clamped to the rows the cache
 // holds), else the uniform count.
@@ -26,17 +33,16 @@ __device__ inline int64_t tokens_of(int64_t n_uniform, const int32_t* len, int b
   return n < k_rows ? n : k_rows;
 }
 
+// Leaf pass of one CTA: kLeafWarps leaves of head bh (one per warp), then the
+// kSubLevels levels above them that lie inside this group, from shared memory.
 template <typename T, int D>
-__global__ void __launch_bounds__(kLeafWarps * 32) pyramid_leaf_kernel(const T* __restrict__ k, float* __restrict__ pyr,
-                                                                       Layout lay, int64_t n_uniform,
-                                                                       const int32_t* __restrict__ len, int H,
-                                                                       int64_t k_rows, int C, PageMap pm) {
-  __shared__ __align__(16) float sm[2][kLeafWarps][D];
-  const int bh = blockIdx.y;
+__device__ void leaf_group(const T* __restrict__ k, float* pyr, const Layout& lay, int64_t n_uniform,
+                           const int32_t* __restrict__ len, int H, int64_t k_rows, int C, const PageMap& pm, int bh,
+                           int64_t group, float (*sm)[kUpperNodes][D]) {
   const int b = bh / H;
   const int64_t n = tokens_of(n_uniform, len, b, k_rows);
   const int64_t M1 = level_size(n, C, 1);
-  const int64_t leaf0 = static_cast<int64_t>(blockIdx.x) * kLeafWarps;
+  const int64_t leaf0 = group * kLeafWarps;
   if (n <= 0 || leaf0 >= M1) return;
   const int L = num_levels(n, C);
   const int warp = threadIdx.x >> 5;
@@ -56,7 +62,6 @@ __global__ void __launch_bounds__(kLeafWarps * 32) pyramid_leaf_kernel(const T* 
     }
     LeafMean<T, D>::store(mean, &sm[0][warp][0], pbh + (lay.off[1] + leaf) * D, lane);
   }
-  // Levels above the leaves that lie inside this CTA's subtree.
   int cur = 0;
   for (int l = 2; l <= 1 + kSubLevels && l <= L; ++l) {
     __syncthreads();
@@ -78,25 +83,24 @@ __global__ void __launch_bounds__(kLeafWarps * 32) pyramid_leaf_kernel(const T* 
   }
 }
 
-// Folds kUpperNodes nodes of level `la` per CTA into levels la+1 .. la+kUpperLevels.
+// Upper pass of one CTA: kUpperNodes nodes of level la of head bh, folded into
+// levels la+1 .. la+kUpperLevels. Level la was written by other CTAs before a
+// grid-wide barrier, so it is read through L2 (__ldcg), not the read-only path.
 template <int D>
-__global__ void __launch_bounds__(256) pyramid_upper_kernel(float* __restrict__ pyr, Layout lay, int64_t n_uniform,
-                                                            const int32_t* __restrict__ len, int H, int64_t k_rows,
-                                                            int C, int la) {
-  __shared__ __align__(16) float sm[2][kUpperNodes][D];
-  const int bh = blockIdx.y;
+__device__ void upper_group(float* pyr, const Layout& lay, int64_t n_uniform, const int32_t* __restrict__ len, int H,
+                            int64_t k_rows, int C, int la, int bh, int64_t group, float (*sm)[kUpperNodes][D]) {
   const int b = bh / H;
   const int64_t n = tokens_of(n_uniform, len, b, k_rows);
   if (n <= 0) return;
   const int L = num_levels(n, C);
   if (la >= L) return;
   const int64_t Ma = level_size(n, C, la);
-  const int64_t node0 = static_cast<int64_t>(blockIdx.x) * kUpperNodes;
+  const int64_t node0 = group * kUpperNodes;
   if (node0 >= Ma) return;
   float* pbh = pyr + static_cast<int64_t>(bh) * lay.R * D;
   for (int x = threadIdx.x; x < kUpperNodes * D; x += blockDim.x) {
     const int j = x / D, e = x % D;
-    sm[0][j][e] = (node0 + j < Ma) ? pbh[(lay.off[la] + node0 + j) * D + e] : 0.f;
+    sm[0][j][e] = (node0 + j < Ma) ? __ldcg(pbh + (lay.off[la] + node0 + j) * D + e) : 0.f;
   }
   int cur = 0;
   for (int l = la + 1; l <= la + kUpperLevels && l <= L; ++l) {
@@ -118,24 +122,64 @@ __global__ void __launch_bounds__(256) pyramid_upper_kernel(float* __restrict__ 
   }
 }
 
+// The whole pyramid in one cooperative launch. Every CTA walks leaf groups
+// grid-strided; after a grid-wide barrier the upper passes fold the level
+// kSubLevels + 1 nodes kUpperLevels levels at a time, with a barrier between
+// passes. n_max bounds every head's token count, so all CTAs take the same
+// number of barriers.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) pyramid_kernel(const T* __restrict__ k, float* pyr, Layout lay,
+                                                           int64_t n_max, int64_t n_uniform,
+                                                           const int32_t* __restrict__ len, int H, int BH,
+                                                           int64_t k_rows, int C, PageMap pm) {
+  __shared__ __align__(16) float sm[2][kUpperNodes][D];
+  const int64_t groups = (level_size(n_max, C, 1) + kLeafWarps - 1) / kLeafWarps;
+  for (int64_t u = blockIdx.x; u < groups * BH; u += gridDim.x) {
+    leaf_group<T, D>(k, pyr, lay, n_uniform, len, H, k_rows, C, pm, static_cast<int>(u / groups), u % groups, sm);
+    __syncthreads();
+  }
+  const int L = num_levels(n_max, C);
+  for (int la = 1 + kSubLevels; la < L; la += kUpperLevels) {
+    cg::this_grid().sync();
+    const int64_t ng = (level_size(n_max, C, la) + kUpperNodes - 1) / kUpperNodes;
+    for (int64_t u = blockIdx.x; u < ng * BH; u += gridDim.x) {
+      upper_group<D>(pyr, lay, n_uniform, len, H, k_rows, C, la, static_cast<int>(u / ng), u % ng, sm);
+      __syncthreads();
+    }
+  }
+}
+
+int resident_ctas(const void* kern) {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  return per_sm * sms;
+}
+
 template <typename T, int D>
 cudaError_t build_impl(const void* k, float* pyr, const Layout& lay, int64_t n_max, int64_t n_uniform,
                        const int32_t* len, int BH, int H, int64_t k_rows, int C, PageMap pm, cudaStream_t st) {
-  const int64_t M1 = level_size(n_max, C, 1);
-  dim3 grid(static_cast<unsigned>((M1 + kLeafWarps - 1) / kLeafWarps), BH);
-  pyramid_leaf_kernel<T, D><<<grid, kLeafWarps * 32, 0, st>>>(static_cast<const T*>(k), pyr, lay, n_uniform, len, H,
-                                                               k_rows, C, pm);
-  count_launch();
-  cudaError_t err = cudaGetLastError();
-  const int L = num_levels(n_max, C);
-  for (int la = 1 + kSubLevels; la < L && err == cudaSuccess; la += kUpperLevels) {
-    const int64_t Ma = level_size(n_max, C, la);
-    dim3 g2(static_cast<unsigned>((Ma + kUpperNodes - 1) / kUpperNodes), BH);
-    pyramid_upper_kernel<D><<<g2, 256, 0, st>>>(pyr, lay, n_uniform, len, H, k_rows, C, la);
-    count_launch();
-    err = cudaGetLastError();
+  const int64_t groups = (level_size(n_max, C, 1) + kLeafWarps - 1) / kLeafWarps * BH;
+  const void* kern = reinterpret_cast<const void*>(pyramid_kernel<T, D>);
+  const int64_t cap = resident_ctas(kern);
+  const unsigned grid = static_cast<unsigned>(groups < cap ? groups : cap);
+  const T* kp = static_cast<const T*>(k);
+  void* args[] = {&kp, &pyr, const_cast<Layout*>(&lay), &n_max, &n_uniform, &len, &H, &BH, &k_rows, &C, &pm};
+  cudaError_t err;
+  {
+    TimedLaunch tl("pyramid_kernel", st);
+    err = cudaLaunchCooperativeKernel(kern, dim3(grid), dim3(kThreads), args, 0, st);
   }
-  return err;
+  count_launch();
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
 }
 
 }  // namespace

@@ -31,21 +31,26 @@ struct LeafMean {
   }
 };
 
-__device__ inline void add16(const float* p, float* acc) {
-  float4 v = *reinterpret_cast<const float4*>(p);
-  acc[0] += v.x;
-  acc[1] += v.y;
-  acc[2] += v.z;
-  acc[3] += v.w;
+// Adds 16 bytes of key elements (4 fp32 or 8 bf16), already loaded, to acc.
+__device__ inline void add16(uint4 u, const float*, float* acc) {
+  acc[0] += __uint_as_float(u.x);
+  acc[1] += __uint_as_float(u.y);
+  acc[2] += __uint_as_float(u.z);
+  acc[3] += __uint_as_float(u.w);
 }
-__device__ inline void add16(const bf16* p, float* acc) {
-  uint4 u = *reinterpret_cast<const uint4*>(p);
+__device__ inline void add16(uint4 u, const bf16*, float* acc) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     acc[2 * i] += __uint_as_float(w[i] << 16);
     acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
   }
+}
+// Plain (coherent) loads: callers may read rows that the same kernel has just
+// written, or rows in shared memory.
+template <typename T>
+__device__ inline void add16(const T* p, float* acc) {
+  add16(*reinterpret_cast<const uint4*>(p), p, acc);
 }
 
 // Mean of key rows [lo, hi) of one head (rows of D elements), computed by one
@@ -61,7 +66,16 @@ __device__ inline void leaf_mean_warp(const T* __restrict__ kbh, int64_t lo, int
 #pragma unroll
   for (int e = 0; e < LM::kVec; ++e) acc[e] = 0.f;
   int64_t j = lo + lane / LM::kLpr;
-#pragma unroll 4
+  // Batches of kBatch loads in flight, then their adds in row order (the
+  // summation order is that of a plain row-by-row loop).
+  constexpr int kBatch = 8;
+  for (; j + (kBatch - 1) * LM::kRpw < hi; j += kBatch * LM::kRpw) {
+    uint4 u[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) u[i] = *reinterpret_cast<const uint4*>(kbh + (j + i * LM::kRpw) * D + col);
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) add16(u[i], kbh, acc);
+  }
   for (; j < hi; j += LM::kRpw) add16(kbh + j * D + col, acc);
 #pragma unroll
   for (int o = LM::kLpr; o < 32; o <<= 1)

@@ -170,6 +170,7 @@ cudaError_t launch_select_rows(const PrefillArgs& a, const void* q, const void* 
   return dispatch_tdg(a.dtype, a.d, a.H_q / a.H_kv, [&](auto tt, auto dd, auto gg) -> cudaError_t {
     using T = typename decltype(tt)::type;
     constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
+    TimedLaunch tl("select_rows_kernel", st);
     select_rows_kernel<T, D, G><<<row_blocks(a), kRowWarps * 32, 0, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), pyr, lay, a, sel, sel_score);
     count_launch();
@@ -182,6 +183,7 @@ cudaError_t launch_attn_rows(const PrefillArgs& a, const void* q, const void* k,
   return dispatch_tdg(a.dtype, a.d, a.H_q / a.H_kv, [&](auto tt, auto dd, auto gg) -> cudaError_t {
     using T = typename decltype(tt)::type;
     constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
+    TimedLaunch tl("attn_rows_kernel", st);
     attn_rows_kernel<T, D, G><<<row_blocks(a), kRowWarps * 32, 0, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), sel, a, static_cast<T*>(out),
         lse);
@@ -195,6 +197,7 @@ cudaError_t launch_flat_rows(const PrefillArgs& a, const void* q, const float* p
   return dispatch_tdg(a.dtype, a.d, a.H_q / a.H_kv, [&](auto tt, auto dd, auto gg) -> cudaError_t {
     using T = typename decltype(tt)::type;
     constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
+    TimedLaunch tl("flat_rows_kernel", st);
     flat_rows_kernel<T, D, G><<<row_blocks(a), kRowWarps * 32, 0, st>>>(static_cast<const T*>(q), pyr, R, a, sel);
     count_launch();
     return cudaGetLastError();
@@ -205,6 +208,7 @@ cudaError_t launch_exact_rows(const PrefillArgs& a, const void* q, const void* k
   return dispatch_tdg(a.dtype, a.d, a.H_q / a.H_kv, [&](auto tt, auto dd, auto gg) -> cudaError_t {
     using T = typename decltype(tt)::type;
     constexpr int D = decltype(dd)::value, G = decltype(gg)::value;
+    TimedLaunch tl("exact_rows_kernel", st);
     exact_rows_kernel<T, D, G><<<row_blocks(a), kRowWarps * 32, 0, st>>>(static_cast<const T*>(q),
                                                                           static_cast<const T*>(k), a, sel);
     count_launch();

@@ -586,23 +586,34 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
     const int64_t n4 = static_cast<int64_t>(a.B) * a.H_kv * lay.R * a.d / 4;
     const int64_t gb = (n4 + 255) / 256;
     const unsigned g = static_cast<unsigned>(gb < sm_count() * 16 ? gb : sm_count() * 16);
+    TimedLaunch tl("split_kernel", st);
     split_kernel<<<g, 256, 0, st>>>(reinterpret_cast<const float4*>(pyr), ws.planes, n4);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
     constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
+    TimedLaunch tl("router_kernel", st);
     router_kernel<D, GG><<<static_cast<unsigned>((rows + kRouterWarps - 1) / kRouterWarps), kRouterWarps * 32, 0,
                            st>>>(static_cast<const bf16*>(q), pyr, lay, a, ws, sel, sel_score);
     count_launch();
     return cudaGetLastError();
   });
   if (e != cudaSuccess) return e;
-  scan_kernel<<<1, 1024, 0, st>>>(ws, nb);
+  {
+    TimedLaunch tl("scan_kernel", st);
+    scan_kernel<<<1, 1024, 0, st>>>(ws, nb);
+  }
   count_launch();
-  scatter_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(ws, rows, a.Nq, M1);
+  {
+    TimedLaunch tl("scatter_kernel", st);
+    scatter_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(ws, rows, a.Nq, M1);
+  }
   count_launch();
-  itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(ws, nb, M1);
+  {
+    TimedLaunch tl("itemize_kernel", st);
+    itemize_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(ws, nb, M1);
+  }
   count_launch();
   if (leaf_umma_supported(a)) {
     if ((e = launch_leaf_umma(a, q, k, ws, nb, M1, st)) != cudaSuccess) return e;
@@ -625,6 +636,7 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLeafThreads, smem) != cudaSuccess ||
             per_sm < 1)
           per_sm = 1;
+        TimedLaunch tl("leaf_kernel", st);
         kern<<<static_cast<unsigned>(sm_count() * per_sm), kLeafThreads, smem, st>>>(tmq, tmk, a, ws, nb, M1, faults);
         count_launch();
         return cudaGetLastError();
@@ -633,7 +645,10 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
     });
     if (e != cudaSuccess) return e;
   }
-  final_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(a, ws, sel, sel_score, rows);
+  {
+    TimedLaunch tl("final_kernel", st);
+    final_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(a, ws, sel, sel_score, rows);
+  }
   count_launch();
   return cudaGetLastError();
 }

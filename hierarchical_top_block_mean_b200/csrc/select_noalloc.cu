@@ -29,20 +29,42 @@ static __device__ __align__(256) unsigned char g_select_scratch[kScratchBytes];
 constexpr int kMaxDevices = 128;
 std::mutex g_setup_mu;
 void* g_scratch_dev[kMaxDevices] = {};
+void* g_scratch_ctx[kMaxDevices] = {};  // the context each cached address belongs to
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+// The current driver context (CUcontext) as an opaque handle, fetched through
+// the runtime's driver entry point so that the library need not link libcuda.
+void* current_context() {
+  using Fn = int (*)(void**);
+  static Fn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<Fn>(p);
+  }();
+  void* ctx = nullptr;
+  if (fn == nullptr || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of the scratch array on the current device. It is looked up
+// with cudaGetSymbolAddress on the first call per device, with that device
+// current, and cached. A new context on that device (after cudaDeviceReset
+// the module is loaded again, possibly elsewhere) triggers a fresh lookup.
 cudaError_t scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_dev[dev] == nullptr) {
+  if (g_scratch_dev[dev] == nullptr || ctx == nullptr || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_select_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_dev[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_dev[dev];
   return cudaSuccess;

@@ -73,6 +73,8 @@ class SeqParallelPrefill:
         self.rank = dist.get_rank(group)
         self.q0, self.n = shard_span(pr.N, self.world, self.rank)
         dev = torch.device(device)
+        if dev.type == "cuda" and shard is None and dev.index is not None:
+            torch.cuda.set_device(dev)  # the library launches on the current device
         self._kernels = shard is None  # the default shard runs the library's CUDA kernels
         self.shard = PrefillShard(pr, self.q0, self.n, dev) if shard is None else shard
         self.k_full = torch.empty((pr.B, pr.H_kv, pr.N, pr.d), dtype=pr.dtype, device=dev)

@@ -15,7 +15,8 @@
  *   - Pointers named q, k, v, pyr, sel, out, lse, ws, k_cache, v_cache, len,
  *     status are DEVICE pointers to memory the caller owns. The library never
  *     allocates, never synchronises the device and keeps no state between
- *     calls (except the launch counter of pisa_launch_count).
+ *     calls (except the launch counter of pisa_launch_count, the records of
+ *     pisa_timing_start/stop and the scratch of pisa_select_noalloc).
  *   - Tensors are dense and row-major: q [B, H_q, N, d]; k, v [B, H_kv, N, d];
  *     query head h' belongs to kv head h' / G_Q with G_Q = H_q / H_kv.
  *   - dtype selects the storage of q, k, v and out: PISA_DTYPE_BF16 or
@@ -91,6 +92,27 @@ uint64_t pisa_launch_count(void);
 uint64_t pisa_device_faults(void);
 
 /*
+ * Per-kernel timing for profiling. Not part of the method; a measurement aid.
+ * After pisa_timing_start(), every kernel this library launches (on any
+ * stream, from any entry point) is bracketed by two CUDA events recorded on
+ * its launching stream, until pisa_timing_stop(). Each bracketed launch
+ * creates two events, so keep timing windows short and off the hot path of
+ * production runs; outside a window the cost is one atomic load per launch.
+ *   pisa_timing_start: clears earlier records and turns timing on.
+ *   pisa_timing_stop: turns timing off, waits for the recorded events (this
+ *     synchronises with every stream that was timed), and writes up to
+ *     max_kernels entries, one per kernel name in first-launch order:
+ *     names[i] (a static string owned by the library), total_ms[i] (sum of
+ *     event durations) and launches[i]. Any array may be NULL. Returns the
+ *     number of distinct kernel names (which may exceed max_kernels), or -1
+ *     if an event failed (the records are dropped either way).
+ * Kernels overlapping on several streams are each timed from their own
+ * stream's events, so their durations include any time shared with others.
+ */
+pisa_status pisa_timing_start(void);
+int pisa_timing_stop(int max_kernels, const char** names, double* total_ms, int* launches);
+
+/*
  * Pyramid geometry (host only, pure integer arithmetic) — §Pyramid level
  * sizes: M_0 = N, M_1 = ceil(N / C), M_{l+1} = ceil(M_l / g) until M_L = 1.
  * Writes L to *num_levels. If level_offsets is not NULL it receives L + 1
@@ -138,11 +160,19 @@ pisa_status pisa_select(const pisa_config* cfg, const void* q, const void* k, co
  * Flat single-level selection — §BSA: a flat method scores all M = ceil(N/C)
  * leaf summaries per query. Score reading: u_i = sum over the group of
  * scale * q_{h',t} . kbar^{(1)}_i; top K with the same validity, tie, order
- * and padding rules as pisa_select. Needs no workspace.
+ * and padding rules as pisa_select.
  *   q : [B, H_q, N, d];  pyr : [B, H_kv, R, d] (only level 1 is read);
  *   sel : [B, H_kv, N, K] int32.
+ *   ws : device scratch of at least pisa_select_flat_workspace_bytes(cfg)
+ *        bytes, 256-byte aligned, caller-owned, contents on entry ignored
+ *        (bf16 with d = 128 needs it: the group-summed queries and the leaf
+ *        summaries, each split into bf16 hi and lo planes; otherwise the size
+ *        is 0 and ws may be NULL). Too small a ws returns PISA_ERR_WORKSPACE
+ *        before anything is enqueued.
  */
-pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float* pyr, int32_t* sel, void* stream);
+size_t pisa_select_flat_workspace_bytes(const pisa_config* cfg);
+pisa_status pisa_select_flat(const pisa_config* cfg, const void* q, const float* pyr, int32_t* sel, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /*
  * Exact-score flat selection — the single-level block selection that the
@@ -191,6 +221,8 @@ pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const vo
  *   - Calls no cudaMalloc or cudaFree and allocates nothing.
  *   - The first call on each device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     A call in a new context on that device (after cudaDeviceReset) looks it
+ *     up again, so it too should come before any capture.
  *   - All calls in the process share the one array per device: calls whose
  *     execution overlaps on the GPU (different streams, or different host
  *     threads without ordering) race on it and give wrong selections. Order

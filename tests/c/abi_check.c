@@ -42,5 +42,12 @@ int main(void) {
   cfg.K = 17;
   check(pisa_sparse_attn_fwd(&cfg, p, p, p, p, p, NULL, NULL) == PISA_ERR_UNSUPPORTED, "K = 17 unsupported");
   check(pisa_launch_count() == before, "nothing launched");
+
+  /* An empty timing window needs no device and records nothing. */
+  const char* names[4];
+  double ms[4];
+  int launches[4];
+  check(pisa_timing_start() == PISA_OK, "timing start");
+  check(pisa_timing_stop(4, names, ms, launches) == 0, "empty timing window");
   return failed;
 }

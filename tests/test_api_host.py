@@ -66,12 +66,13 @@ def test_invalid_configs_rejected_before_launch(kw, code):
     cfg = _cfg(**kw)
     assert lib.pisa_build_pyramid(ctypes.byref(cfg), dummy, dummy, None) == code
     assert lib.pisa_select(ctypes.byref(cfg), dummy, dummy, dummy, dummy, None, dummy, 1 << 30, None) == code
-    assert lib.pisa_select_flat(ctypes.byref(cfg), dummy, dummy, dummy, None) == code
+    assert lib.pisa_select_flat(ctypes.byref(cfg), dummy, dummy, dummy, dummy, 1 << 30, None) == code
     assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), dummy, dummy, dummy, dummy, dummy, None, None) == code
     assert lib.pisa_select_exact(ctypes.byref(cfg), dummy, dummy, dummy, None) == code
     assert lib.pisa_sparse_attn_bwd(ctypes.byref(cfg), dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy,
                                     dummy, dummy, 1 << 30, None) == code
     assert lib.pisa_select_workspace_bytes(ctypes.byref(cfg)) == 0
+    assert lib.pisa_select_flat_workspace_bytes(ctypes.byref(cfg)) == 0
     assert lib.pisa_attn_bwd_workspace_bytes(ctypes.byref(cfg)) == 0
     assert lib.pisa_launch_count() == before
 
@@ -167,4 +168,23 @@ def test_header_compiles_as_c99_and_links(tmp_path):
                     "-Wl,-rpath," + lib_dir, "-o", exe], check=True, capture_output=True, text=True)
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
-    assert "FAIL" not in r.stdout and r.stdout.count("ok ") == 13, r.stdout
+    assert "FAIL" not in r.stdout and r.stdout.count("ok ") == 15, r.stdout
+
+
+def test_flat_workspace_sized_and_checked_before_launch():
+    # bf16 with d = 128 takes the tensor-core flat selector, whose hi/lo
+    # operand planes live in the caller's workspace: 2 x (B H_kv N + B H_kv M_1)
+    # rows of 128 bf16, each plane 256-byte aligned. Too small a workspace is
+    # refused before anything is enqueued; other shapes need none.
+    lib = _lib.lib()
+    cfg = _cfg(N=1000, H_q=8, H_kv=2, d=128, C=64)
+    need = lib.pisa_select_flat_workspace_bytes(ctypes.byref(cfg))
+    rows_q, rows_k = 2 * 1000, 2 * 16
+    al = lambda x: (x + 255) // 256 * 256
+    assert need == 2 * al(rows_q * 256) + 2 * al(rows_k * 256)
+    before = lib.pisa_launch_count()
+    dummy = ctypes.c_void_p(256)
+    assert lib.pisa_select_flat(ctypes.byref(cfg), dummy, dummy, dummy, dummy, need - 1, None) == 3
+    assert lib.pisa_select_flat(ctypes.byref(cfg), dummy, dummy, dummy, None, need, None) == 3
+    assert lib.pisa_launch_count() == before
+    assert lib.pisa_select_flat_workspace_bytes(ctypes.byref(_cfg(N=1000, d=64, C=32))) == 0

@@ -136,3 +136,13 @@ def test_paged_state_refuses_out_of_pool_pages(calls):
     with pytest.raises(ValueError):
         ok.check_block_table()
     assert calls == []
+
+
+def test_tensor_on_another_device_is_refused(monkeypatch):
+    # The library launches on the current device; a tensor on another GPU
+    # (or tensors of one call spread over GPUs) must be refused before the C
+    # call. The current device is stubbed to cuda:0.
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    api._check_device_index(0, "q")
+    with pytest.raises(ValueError, match="cuda:1"):
+        api._check_device_index(1, "k")

@@ -54,3 +54,34 @@ def test_cpu_decode_baseline_on_a_small_decode_workload():
     r = bench.cpu_decode_baseline(wd, budget_s=1.0)
     assert r["kind"] == "oracle" and r["us_per_step"] > 0 and r["cores"] >= 1
     assert "3 steps" in r["sample"] and "701 tokens" in r["sample"]
+
+
+def test_work_model_matches_the_oracle_trace(oracle):
+    """The bench's algorithmic work model counts, per query row, the leaf
+    candidates the search scores and the child summaries the router gathers
+    from the level geometry alone. The oracle's per-level trace gives the true
+    counts: the model may only over-count a block whose second child starts
+    after t, so it stays within a few percent above the truth."""
+    import numpy as np
+    from hierarchical_top_block_mean_b200 import workloads
+    w = workloads.Prefill("model", B=1, N=3000, H_q=4, H_kv=1, d=16, C=16, K=4, causal=True, dtype="f32", seed=3)
+    x = workloads.prefill_inputs(w)
+    cfg = oracle.make_cfg(B=1, N=w.N, H_q=w.H_q, H_kv=w.H_kv, d=w.d, C=w.C, K=w.K, causal=True, dtype_code=0)
+    pyr = oracle.build_pyramid(x["k"], w.C)
+    rows = np.array([(0, 0, t) for t in range(w.N)], np.int64)
+    _, _, tr = oracle.select_rows(cfg, x["q"], x["k"], pyr, rows, trace=True)
+    scored = tr["n"] > w.K
+    pairs = int(np.where(scored[:, 1], tr["n"][:, 1], 0).sum())
+    sizes, _ = oracle.geometry(w.N, w.C)
+    gathered = 0
+    for r, t in enumerate(range(w.N)):
+        for l in range(2, len(sizes)):
+            if scored[r, l]:
+                for s in range(tr["n"][r, l]):
+                    i = tr["cand"][r, l, s]
+                    gathered += sum(1 for c in (2 * i, 2 * i + 1)
+                                    if c < sizes[l - 1] and c * (w.C << (l - 2)) <= t)
+    m = bench.work_model(w)
+    assert pairs <= m["leaf_pairs"] <= 1.05 * pairs
+    assert m["leaf_flops"] == m["leaf_pairs"] * 2 * (w.H_q // w.H_kv) * w.C * w.d
+    assert gathered * w.d * 4 <= m["router_gather_bytes"] <= 1.10 * gathered * w.d * 4

@@ -47,6 +47,11 @@ def _run(w, rows_per_head=None):
     sel_gpu = P.gather_rows(p.sel, rows)
     n, n_ex, bad, bad_ex = P.compare_selection(w, sel_gpu, sel_ref, gap)
     assert bad == 0, f"{w.name}: {bad} non-exempt selection mismatches of {n} rows ({n_ex} exempt)"
+    # Even inside the near-tie exemption the GPU mostly agrees: the kernels'
+    # fp32 scores sit within ~1e-5 of the oracle's, far inside the 1e-3
+    # exemption, so a regression that moved scores would show up as many
+    # exempt rows that differ.
+    assert bad_ex <= max(2, 0.2 * n_ex), f"{w.name}: {bad_ex} of {n_ex} exempt rows differ"
     # Attention with the GPU's own selection, so selection differences cannot hide errors.
     out_ref, lse_ref = O.attn_rows(cfg, qh, kh, vh, rows, sel_gpu)
     err = P.check_attention(w, P.gather_out(w, p.out, rows), P.gather_lse(w, p.lse, rows), out_ref, lse_ref)
@@ -90,8 +95,8 @@ def test_large_K_prefill_equals_dense_attention():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,rows", [("needle_16k", 4096), ("clustered_64k", 2048), ("needle_64k_g8", 2048),
-                                       ("needle_256k", 1024)])
+@pytest.mark.parametrize("name,rows", [("needle_16k", 4096), ("clustered_64k", 8192), ("needle_64k_g8", 4096),
+                                       ("needle_256k", 8192)])
 def test_prefill_parity_full_size(name, rows):
     w = workloads.PREFILL[name]
     r = _run(w, rows)

@@ -7,9 +7,10 @@ exact by construction:
     of equal content have equal summaries at every level and equal scores in
     both fp64 and the kernels' fp32;
   * every key the same vector, so every full block of a level ties.
-Rows are compared without any exemption for exact ties (a level whose K-th
-and (K+1)-th oracle scores are equal). Only a level whose K-th and (K+1)-th
-scores differ by a non-zero amount below 1e-3 exempts its row. The pyramid
+Rows are compared without any exemption for exact ties. A row is exempt only
+where some candidate's oracle score differs from the K-th best by a non-zero
+amount below 1e-3 (rounding could reorder the two; with tied classes that can
+change the kept set even when the K-th and (K+1)-th scores are equal). The pyramid
 search, the flat selector and the exact-score selector are all checked, on
 the tcgen05 (G_Q = 8) and mma.sync (G_Q = 4) leaf paths."""
 import numpy as np
@@ -32,9 +33,19 @@ CASES = [
 ]
 
 
+def _near_kth(scores, K):
+    """True when some candidate's score differs from the K-th best by a
+    non-zero amount below the tie tolerance: rounding could then reorder the
+    two and change the kept set. Exactly equal scores are not near: the tie
+    rule decides them."""
+    s = np.sort(scores)[::-1]
+    d = np.abs(scores - s[K - 1])
+    return bool(((d > 0) & (d < P.GAP_TOL)).any())
+
+
 def _exempt_rows(w, trace):
-    """Rows with a scored level whose K-th and (K+1)-th oracle scores differ by
-    a non-zero amount below the tie tolerance; exact ties are not exempt."""
+    """Rows with a scored level where _near_kth holds, and the number of
+    scored levels whose K-th and (K+1)-th oracle scores tie exactly."""
     n_rows = trace["n"].shape[0]
     ex = np.zeros(n_rows, bool)
     n_tied = 0
@@ -43,15 +54,36 @@ def _exempt_rows(w, trace):
             n = trace["n"][r, l]
             if n <= w.K:
                 continue
-            s = np.sort(trace["score"][r, l, :n])[::-1]
-            g = s[w.K - 1] - s[w.K]
-            n_tied += g == 0
-            ex[r] |= 0 < g < P.GAP_TOL
+            sc = trace["score"][r, l, :n]
+            s = np.sort(sc)[::-1]
+            n_tied += s[w.K - 1] == s[w.K]
+            ex[r] |= _near_kth(sc, w.K)
     return ex, n_tied
 
 
-def _flat_like_exempt(gap):
-    return (gap > 0) & (gap < P.GAP_TOL)
+def _leaf_scores(w, x, pyr_ref, rows, exact):
+    """fp64 scores of every usable leaf for each row, used only to decide which
+    rows a rounding-level reordering could change: the exact raw-key block
+    LSE summed over the group (exact) or the group-summed dot product with the
+    leaf mean (flat)."""
+    G = w.H_q // w.H_kv
+    M1 = -(-w.N // w.C)
+    out = []
+    for (b, h, t) in rows:
+        q = x["q"][b, h * G:(h + 1) * G, t, :].double()
+        nv = min(M1, t // w.C + 1) if w.causal else M1
+        if exact:
+            k = x["k"][b, h].double()
+            lg = (q @ k.T) / np.sqrt(w.d)
+            if w.causal:
+                lg[:, t + 1:] = -np.inf
+            pad = torch.full((G, M1 * w.C - w.N), -np.inf, dtype=lg.dtype)
+            u = torch.logsumexp(torch.cat([lg, pad], 1).reshape(G, M1, w.C), 2).sum(0)
+        else:
+            leaves = torch.from_numpy(pyr_ref[b, h, :M1])
+            u = (q.sum(0) @ leaves.T) / np.sqrt(w.d)
+        out.append(u[:nv].numpy())
+    return out
 
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
@@ -75,10 +107,13 @@ def test_exact_ties_go_to_the_lower_block_index(w):
     bad = ~same & ~ex
     assert not bad.any(), f"{w.name}: {bad.sum()} rows differ ({ex.sum()} exempt of {len(rows)}); " \
                           f"first at t={rows[np.argmax(bad), 2]}"
+    xh = dict(q=qh, k=kh)
     for name, got, (ref, gap) in (("flat", flat, O.select_flat_rows(cfg, qh, pyr_ref, rows)),
                                   ("exact", exact, O.select_exact_rows(cfg, qh, kh, rows))):
+        scores = _leaf_scores(w, xh, pyr_ref, rows, exact=name == "exact")
+        ex = np.array([len(u) > w.K and _near_kth(u, w.K) for u in scores])
         same = (P.gather_rows(got, rows) == ref).all(1)
-        bad = ~same & ~_flat_like_exempt(gap)
+        bad = ~same & ~ex
         assert not bad.any(), f"{w.name} {name}: {bad.sum()} rows differ; first at t={rows[np.argmax(bad), 2]}"
         assert (gap == 0).sum() > len(rows) // 4, f"{w.name} {name}: too few exact ties"
     if w.period == 1:

@@ -15,8 +15,10 @@ import torch
 from hierarchical_top_block_mean_b200 import _lib, api, workloads
 
 
-def _inputs(seed):
-    w = workloads.PREFILL["needle_16k"].with_(name=f"noalloc_{seed}", N=3000, n_needles=8, seed=seed)
+def _inputs(seed, **kw):
+    base = dict(name=f"noalloc_{seed}", N=3000, n_needles=8, seed=seed)
+    base.update(kw)
+    w = workloads.PREFILL["needle_16k"].with_(**base)
     x = workloads.prefill_inputs(w, device=torch.device("cuda"))
     return w, x
 
@@ -41,8 +43,11 @@ def _with_workspace(w, x, pyr):
 
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_select_on_two_calls():
-    for seed in (6101, 6102):  # two calls in a row, different inputs, one shared scratch array
-        w, x = _inputs(seed)
+    # Two calls in a row, different inputs, one shared scratch array. The
+    # first has G_Q = 4 (mma.sync leaf scorer); the second G_Q = 8 with
+    # d = 128, C = 64, which takes the tcgen05 leaf scorer and its work lists.
+    for seed, kw in ((6101, {}), (6102, dict(H_q=16, H_kv=2, N=3100))):
+        w, x = _inputs(seed, **kw)
         pyr = api.build_pyramid(x["k"], C=w.C)
         want_sel, want_score = _with_workspace(w, x, pyr)
         got_sel, got_score = _noalloc(w, x, pyr)
