@@ -12,16 +12,16 @@
 //
 // flat_umma_kernel: one CTA per (kv head, tile of 128 queries); the tile's
 // hi and lo rows stay in shared memory as the A operands.
-//   warp 4, one lane (loads): the hi and lo planes of each 64-leaf tile by
+//   warp 16, one lane (loads): the hi and lo planes of each 64-leaf tile by
 //     bulk tensor copy into a ring of kFlStages buffers;
-//   warp 5, one lane (MMA): per leaf tile, 3 x 8 tcgen05.mma (M = 128
+//   warp 17, one lane (MMA): per leaf tile, 3 x 8 tcgen05.mma (M = 128
 //     queries, N = 64 leaves, K = 16) into a ring of TMEM accumulators, then
 //     commits that free the leaf buffer and publish the accumulator;
-//   warps 0-3 (epilogue): warp w reads TMEM lane quarter w; each thread owns
-//     one query, loads its 64 scores, and keeps its running top-K list in
-//     registers: a score enters only if it ranks before the list's K-th
-//     (leaves are visited in ascending order, so an equal score from a later
-//     leaf loses the tie).
+//   warps 0-15 (epilogue): four warps per TMEM lane quarter, 8 query rows
+//     each; a warp walks its rows two at a time (one per half-warp) testing
+//     64 leaves per row at once against the row's K-th best, and merges the
+//     rare entrants into the row's running top-K list with a half-warp
+//     sorted insert.
 // Causal tiles stop at the last leaf their latest query can use and are
 // launched longest first. Every mbarrier wait is bounded in time; the TMEM
 // allocation is always released before exit.
@@ -35,7 +35,7 @@ namespace pisa {
 
 namespace {
 
-constexpr int kFlEpiWarps = 4;
+constexpr int kFlEpiWarps = 16;
 constexpr int kFlLoadWarp = kFlEpiWarps;
 constexpr int kFlMmaWarp = kFlEpiWarps + 1;
 constexpr int kFlThreads = 32 * (kFlEpiWarps + 2);
@@ -44,8 +44,9 @@ constexpr int kFlAccStages = 4;                // TMEM accumulators of 64 column
 constexpr uint32_t kFlTmemCols = kFlAccStages * 64;
 constexpr int kFlQBytes = 128 * 128 * 2;       // 128 queries x 128 bf16, two 64-column halves
 constexpr int kFlLeafBytes = 64 * 128 * 2;     // 64 leaves x 128 bf16, two 64-column halves
-constexpr int kFlLists = 128 * kMaxK * 4;      // per query: kMaxK leaves for the final sort
-constexpr int kFlSmem = 1024 + 2 * kFlQBytes + kFlStages * 2 * kFlLeafBytes + kFlLists;
+constexpr int kFlLists = 128 * kMaxK * 8;      // per query: kMaxK (score, leaf) entries
+constexpr int kFlStage = kFlEpiWarps * 8 * 64 * 4;   // per epilogue warp: 8 rows x 64 scores
+constexpr int kFlSmem = 1024 + 2 * kFlQBytes + kFlStages * 2 * kFlLeafBytes + kFlLists + kFlStage;
 
 // Workspace: q hi, q lo [B H_kv N][128]; leaf hi, leaf lo [B H_kv M1][128] (bf16).
 struct FlatWs {
@@ -133,7 +134,9 @@ __global__ void __launch_bounds__(kFlThreads, 1)
   unsigned char* qhi = smem;                         // A operands, resident
   unsigned char* qlo = smem + kFlQBytes;
   unsigned char* lbuf = smem + 2 * kFlQBytes;        // [kFlStages][hi, lo][kFlLeafBytes]
-  int* li = reinterpret_cast<int*>(lbuf + kFlStages * 2 * kFlLeafBytes);  // [128][kMaxK] final sort of kept leaves
+  float* ls = reinterpret_cast<float*>(lbuf + kFlStages * 2 * kFlLeafBytes);  // [128][kMaxK] kept scores
+  int* li = reinterpret_cast<int*>(ls + 128 * kMaxK);                          // [128][kMaxK] kept leaves
+  float* stage_buf = reinterpret_cast<float*>(li + 128 * kMaxK);              // [16 warps][8][64] scores
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool causal = a.causal != 0;
@@ -160,6 +163,10 @@ __global__ void __launch_bounds__(kFlThreads, 1)
   if (warp == 0) {
     tmem_alloc(&tmem_base_sh, kFlTmemCols);
     tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < 128 * kMaxK; i += blockDim.x) {
+    ls[i] = -INFINITY;
+    li[i] = INT_MAX;
   }
   tc_fence_before();
   __syncthreads();
@@ -213,22 +220,29 @@ __global__ void __launch_bounds__(kFlThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    // Each thread keeps its query's best K (score, leaf) pairs in registers,
-    // worst first: rs[0] is the K-th best, the entry a new score must beat.
-    // Slots K .. kMaxK-1 hold +inf sentinels that nothing passes, so the list
-    // never needs a dynamic index. A new entry replaces rs[0] and rises by
-    // a fixed sequence of compare-and-swaps.
-    const int row = 32 * warp + lane;  // TMEM lane = query t0 + row
-    const int64_t t = t0 + row;
-    const bool qok = t < N;
-    const int64_t lim = !qok ? 0 : (causal ? (t / a.C + 1 < M1 ? t / a.C + 1 : M1) : M1);
+    // Warp w reads TMEM lane quarter w & 3 and owns 8 of its query rows
+    // (part w >> 2). Its lanes stage those rows' 64 scaled scores in shared
+    // memory; the warp then walks its rows two at a time, one per half-warp,
+    // each lane testing four leaves against the row's K-th best (a ballot
+    // skips row pairs with no new entrant, the usual case). A row's running
+    // top-K list lives in shared memory, one entry per lane of its half when
+    // it changes; entrants are merged one at a time by a half-warp sorted
+    // insert, both halves in step. Ranking is by score, then lower leaf
+    // index, a total order, so the kept set does not depend on the order in
+    // which entrants arrive.
+    const int qtr = warp & 3, part = warp >> 2;
+    const int row0 = 32 * qtr + 8 * part;  // this warp's rows row0 .. row0 + 7
     const int K = a.K;
-    float rs[kMaxK];
-    int ri[kMaxK];
-#pragma unroll
-    for (int p = 0; p < kMaxK; ++p) {
-      rs[p] = p < K ? -INFINITY : INFINITY;
-      ri[p] = p < K ? INT_MAX : -1;
+    const int half = lane >> 4, hl = lane & 15;
+    const unsigned hmask = half ? 0xffff0000u : 0x0000ffffu;
+    float* stg = stage_buf + warp * (8 * 64);  // [8 rows][64 leaves] scaled scores
+    // Lane r < 8 keeps row row0 + r's K-th best (thr, thri) and usable-leaf limit.
+    float thr = -INFINITY;
+    int thri = INT_MAX;
+    int lim = 0;
+    if (lane < 8) {
+      const int64_t t = t0 + row0 + lane;
+      lim = static_cast<int>(t >= N ? 0 : (causal ? (t / a.C + 1 < M1 ? t / a.C + 1 : M1) : M1));
     }
     for (int i = 0; i < ntiles; ++i) {
       const int as = i % kFlAccStages;
@@ -236,50 +250,81 @@ __global__ void __launch_bounds__(kFlThreads, 1)
       __syncwarp();  // the TMEM loads below are warp-collective
       tc_fence_after();
       uint32_t v[64];
-      tmem_ld_cols<64>(tmem + (static_cast<uint32_t>(32 * warp) << 16) + as * 64, v);
+      tmem_ld_cols<64>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + as * 64, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accempty[as]);
-      const int64_t c0 = static_cast<int64_t>(i) * 64;
-      const int nvalid = static_cast<int>(lim - c0 < 0 ? 0 : (lim - c0 > 64 ? 64 : lim - c0));
+      if ((lane >> 3) == part) {
+        float* dst = stg + (lane & 7) * 64;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float u = __uint_as_float(v[j]) * a.scale;
-        const int leaf = static_cast<int>(c0) + j;
-        if (j < nvalid && ranks_before(u, leaf, rs[0], ri[0])) {
-          rs[0] = u;
-          ri[0] = leaf;
+        for (int j = 0; j < 64; j += 4)
+          *reinterpret_cast<float4*>(dst + j) =
+              make_float4(__uint_as_float(v[j]) * a.scale, __uint_as_float(v[j + 1]) * a.scale,
+                          __uint_as_float(v[j + 2]) * a.scale, __uint_as_float(v[j + 3]) * a.scale);
+      }
+      __syncwarp();
+      const int c0 = i * 64;
+      for (int rp = 0; rp < 4; ++rp) {
+        const int rr = 2 * rp + half;  // this half's row
+        const float4 x4 = *reinterpret_cast<const float4*>(stg + rr * 64 + 4 * hl);
+        const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+        float th = __shfl_sync(kFull, thr, rr);
+        int thi = __shfl_sync(kFull, thri, rr);
+        const int lm = __shfl_sync(kFull, lim, rr);
+        const int col0 = c0 + 4 * hl;
+        unsigned mine = 0;  // this lane's entrants, bit e = leaf col0 + e
 #pragma unroll
-          for (int p = 0; p + 1 < kMaxK; ++p) {
-            const bool up = ranks_before(rs[p], ri[p], rs[p + 1], ri[p + 1]);
-            const float ts = rs[p];
-            const int ti = ri[p];
-            rs[p] = up ? rs[p + 1] : ts;
-            ri[p] = up ? ri[p + 1] : ti;
-            rs[p + 1] = up ? ts : rs[p + 1];
-            ri[p + 1] = up ? ti : ri[p + 1];
+        for (int e = 0; e < 4; ++e)
+          if (col0 + e < lm && ranks_before(xv[e], col0 + e, th, thi)) mine |= 1u << e;
+        if (__ballot_sync(kFull, mine != 0u) == 0u) continue;
+        const int row = row0 + rr;
+        float es = hl < K ? ls[row * kMaxK + hl] : -INFINITY;
+        int ei = hl < K ? li[row * kMaxK + hl] : INT_MAX;
+        for (;;) {
+          const unsigned any = __ballot_sync(kFull, mine != 0u);
+          if (any == 0u) break;
+          const unsigned hany = any & hmask;
+          const bool act = hany != 0u;                // this half still has an entrant
+          const int src = act ? __ffs(hany) - 1 : lane;  // its lowest lane
+          const int e = __ffs(mine | 16u) - 1;         // this lane's lowest entrant (4: none)
+          const float my_s = e == 0 ? xv[0] : (e == 1 ? xv[1] : (e == 2 ? xv[2] : xv[3]));
+          const float cs = __shfl_sync(kFull, my_s, src);
+          const int ci = __shfl_sync(kFull, col0 + e, src);
+          if (lane == src && act) mine &= mine - 1u;
+          const bool live = act && ranks_before(cs, ci, th, thi);  // the list may have moved past it
+          const bool before = live && hl < K && ranks_before(cs, ci, es, ei);
+          const float ps = __shfl_up_sync(kFull, es, 1, 16);
+          const int pi = __shfl_up_sync(kFull, ei, 1, 16);
+          const bool pbefore = __shfl_up_sync(kFull, before, 1, 16) && hl > 0;
+          if (before) {
+            es = pbefore ? ps : cs;
+            ei = pbefore ? pi : ci;
           }
+          th = __shfl_sync(kFull, es, K - 1, 16);
+          thi = __shfl_sync(kFull, ei, K - 1, 16);
+        }
+        if (hl < K) {
+          ls[row * kMaxK + hl] = es;
+          li[row * kMaxK + hl] = ei;
+        }
+        // Lane r (< 8) takes row r's new threshold from the half that owns it.
+        const float th_r = __shfl_sync(kFull, th, (lane & 1) << 4);
+        const int thi_r = __shfl_sync(kFull, thi, (lane & 1) << 4);
+        if (lane < 8 && (lane >> 1) == rp) {
+          thr = th_r;
+          thri = thi_r;
         }
       }
     }
-    if (qok) {
-      // Kept leaves ascending, -1 padded.
-      int* out_l = li + row * kMaxK;
-#pragma unroll
-      for (int p = 0; p < kMaxK; ++p)
-        if (p < K) out_l[p] = ri[p];
-      for (int m = 1; m < K; ++m) {
-        const int x = out_l[m];
-        int p = m;
-        while (p > 0 && out_l[p - 1] > x) {
-          out_l[p] = out_l[p - 1];
-          --p;
-        }
-        out_l[p] = x;
-      }
-      int32_t* out = sel + (bh * N + t) * K;
-      for (int m = 0; m < K; ++m) out[m] = out_l[m] == INT_MAX ? -1 : out_l[m];
+    // Kept leaves ascending, -1 padded.
+    for (int rr = 0; rr < 8; ++rr) {
+      const int row = row0 + rr;
+      const int64_t t = t0 + row;
+      if (t >= N) break;
+      int idx = lane < K ? li[row * kMaxK + lane] : INT_MAX;
+      warp_sort_asc(idx);
+      if (lane < K) sel[(bh * N + t) * K + lane] = idx == INT_MAX ? -1 : idx;
     }
   }
   tc_fence_before();

@@ -103,6 +103,32 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     c.ntiles = (c.p_hi - c.p_lo + kTilePairs - 1) / kTilePairs;
     return c;
   };
+  // Position in this CTA's stream of tiles: items blockIdx.x, + gridDim.x,
+  // ..., each cut into tiles of kTilePairs pairs.
+  struct Stream {
+    int item, tl;
+    Cursor2 c;
+    int4 inf_next;
+  };
+  auto stream_begin = [&]() {
+    Stream st;
+    st.item = blockIdx.x;
+    st.tl = 0;
+    st.c = cursor(st.item, info(st.item));
+    st.inf_next = info(st.item + gridDim.x);
+    return st;
+  };
+  auto stream_next = [&](Stream st) {
+    if (st.item < total && ++st.tl >= st.c.ntiles) {
+      st.item += gridDim.x;
+      st.tl = 0;
+      if (st.item < total) {
+        st.c = cursor(st.item, st.inf_next);
+        st.inf_next = info(st.item + gridDim.x);
+      }
+    }
+    return st;
+  };
 
   if (warp >= kEpiWarps && warp < kMmaWarp) {
     // ---------------------------------------------------------- loads
@@ -112,22 +138,33 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const int64_t head_stride = static_cast<int64_t>(a.Nq) * 128;
     int nq = 0;                        // uses of the query ring so far
     int pend[kLag + 1] = {}, np_head = 0, npend = 0;  // filled stages not yet published (FIFO)
-    int4 inf = info(blockIdx.x);
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
-      const Cursor2 c = cursor(item, inf);
-      inf = info(item + gridDim.x);
+    // Each tile's pair words are loaded one tile ahead, so their latency
+    // hides behind the previous tile's copies.
+    auto tile_words = [&](const Stream& st) -> uint32_t {
+      if (st.item >= total) return 0u;
+      const int p0 = st.c.p_lo + st.tl * kTilePairs;
+      return lane < min(kTilePairs, st.c.p_hi - p0) ? ws.pairs[p0 + lane] : 0u;
+    };
+    Stream sm = stream_begin();
+    uint32_t tw_next = tile_words(sm);
+    while (sm.item < total) {
+      const Stream cur = sm;
+      const uint32_t twv = tw_next;
+      sm = stream_next(sm);
+      tw_next = tile_words(sm);
+      const Cursor2& c = cur.c;
       const int64_t b = c.bh / a.H_kv, h = c.bh % a.H_kv;
       const bf16* qg = q + (b * a.H_q + h * 8) * head_stride;  // head 0 of the group
-      const bf16* qrow0 = qg + g0 * head_stride + jcol * 8;                        // this thread's column of head g0
-      for (int tl = 0; tl < c.ntiles; ++tl) {
+      const bf16* qrow0 = qg + g0 * head_stride + jcol * 8;   // this thread's column of head g0
+      {
         const int qs = nq % kQStages;
-        const int p0 = c.p_lo + tl * kTilePairs;
+        const int p0 = c.p_lo + cur.tl * kTilePairs;
         const int np = min(kTilePairs, c.p_hi - p0);
         // Loader thread (warp lw, lane l): 16-byte column j = l & 15 of head
         // row g0 = 2 lw + (l >> 4) (and g0 + 4 with two loader warps) of every query of the tile,
         // so each copy instruction moves two whole 256-byte rows. The tile's
         // query rows are read once per warp and shared by shuffle.
-        const int tw = lane < np ? static_cast<int>(ws.pairs[p0 + lane] >> 5) : 0;
+        const int tw = static_cast<int>(twv >> 5);
         mbar_wait(&qempty[qs], ((nq / kQStages) & 1) ^ 1, faults);
         const uint32_t qd = smem_u32(qbuf + qs * kQStageBytes);
         const uint32_t d0 = qd + (jcol >> 3) * (kQStageBytes / 2) + g0 * 128 + (((jcol & 7) ^ g0) << 4);
@@ -219,22 +256,35 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const float sl2 = a.scale * 1.4426950408889634f;
     const int qtr = warp & 3, grp = warp >> 2;
     const int row = 32 * qtr + lane;  // TMEM lane = (query, head) row of the tile
+    // This group's tiles are every other tile of the stream; each one's pair
+    // word is loaded one own tile ahead.
+    auto row_word = [&](const Stream& st) -> uint32_t {
+      if (st.item >= total) return 0xffffffffu;
+      const int p = st.c.p_lo + st.tl * kTilePairs + row / 8;
+      return p < st.c.p_hi ? ws.pairs[p] : 0xffffffffu;
+    };
+    Stream sm = stream_begin();
     int na = 0;
-    int item = blockIdx.x;
-    Cursor2 c = cursor(item, info(item));
-    int4 inf_next = info(item + gridDim.x);
-    int tl = 0;
-    while (item < total) {
-      if ((na & 1) == grp) {
-        const int p = c.p_lo + tl * kTilePairs + row / 8;
-        const uint32_t w = p < c.p_hi ? ws.pairs[p] : 0xffffffffu;
+    if (grp == 1) {
+      sm = stream_next(sm);
+      na = 1;
+    }
+    uint32_t w_next = row_word(sm);
+    while (sm.item < total) {
+      const Cursor2 c = sm.c;
+      const uint32_t w = w_next;
+      const int na_cur = na;
+      sm = stream_next(stream_next(sm));
+      na += 2;
+      w_next = row_word(sm);
+      {
         const bool ok = w != 0xffffffffu;
         const int64_t key0 = static_cast<int64_t>(c.leaf) * 64;
         int nv = static_cast<int>(min(static_cast<int64_t>(64), a.N - key0));
         if (causal && ok)  // the pair holds the query's row; its position is q0 + row
           nv = static_cast<int>(min(static_cast<int64_t>(nv), a.q0 + static_cast<int64_t>(w >> 5) - key0 + 1));
-        const int as = na % kAccStages;
-        mbar_wait(&accfull[as], (na / kAccStages) & 1, faults);
+        const int as = na_cur % kAccStages;
+        mbar_wait(&accfull[as], (na_cur / kAccStages) & 1, faults);
         __syncwarp();  // the TMEM load below is warp-collective
         tc_fence_after();
         uint32_t v[kAccCols];
@@ -272,15 +322,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         if (ok && (row & 7) == 0) {
           const int64_t orow = static_cast<int64_t>(c.bh) * a.Nq + static_cast<int64_t>(w >> 5);
           ws.score[orow * 32 + (w & 31)] = u;
-        }
-      }
-      ++na;
-      if (++tl >= c.ntiles) {
-        item += gridDim.x;
-        tl = 0;
-        if (item < total) {
-          c = cursor(item, inf_next);
-          inf_next = info(item + gridDim.x);
         }
       }
     }
