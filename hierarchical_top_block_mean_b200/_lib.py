@@ -65,11 +65,13 @@ SIGNATURES = {
     "pisa_select_exact": (_i32, [_PC, _p, _p, _p, _p]),
     "pisa_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_PC]),
     "pisa_sparse_attn_bwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
-    "pisa_sparse_attn_fwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p]),
+    "pisa_attn_fwd_workspace_bytes": (ctypes.c_size_t, [_PC]),
+    "pisa_sparse_attn_fwd": (_i32, [_PC, _p, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
     "pisa_select_noalloc": (_i32, [_PC, _p, _p, _p, _p, _p, _p]),
     "pisa_select_span_workspace_bytes": (ctypes.c_size_t, [_PC, _PS]),
     "pisa_select_span": (_i32, [_PC, _PS, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
-    "pisa_sparse_attn_fwd_span": (_i32, [_PC, _PS, _p, _p, _p, _p, _p, _p, _p]),
+    "pisa_attn_fwd_span_workspace_bytes": (ctypes.c_size_t, [_PC, _PS]),
+    "pisa_sparse_attn_fwd_span": (_i32, [_PC, _PS, _p, _p, _p, _p, _p, _p, _p, ctypes.c_size_t, _p]),
     "pisa_decode_pyramid_rows": (_i64, [_PD]),
     "pisa_decode_workspace_bytes": (_i64, [_PD]),
     "pisa_decode_init": (_i32, [_PD, _p, _p, _p, _p]),

@@ -231,9 +231,24 @@ def select_exact(q, k, *, C: int, K: int, causal: bool, scale: float = 0.0, out=
     return out
 
 
+def _attn_workspace(cfg, span, device, workspace):
+    """The caller's workspace, or a new one of the size the bucketed
+    attention needs (None when that route does not apply)."""
+    if workspace is not None:
+        _need(workspace, "workspace")
+        return workspace
+    need = int(_lib.lib().pisa_attn_fwd_span_workspace_bytes(ctypes.byref(cfg), ctypes.byref(span)))
+    return torch.empty(need, dtype=torch.uint8, device=device) if need > 0 else None
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def sparse_attn_fwd(q, k, v, sel, *, C: int, causal: bool, scale: float = 0.0, out=None, lse=None,
-                    want_lse: bool = True):
-    """Block-sparse attention over the selected leaf blocks: (out [B,H_q,N,d], lse [B,H_q,N] or None)."""
+                    want_lse: bool = True, workspace=None):
+    """Block-sparse attention over the selected leaf blocks: (out [B,H_q,N,d], lse [B,H_q,N] or None).
+    The bucketed route's scratch is allocated here unless `workspace` is given."""
     _need(q, "q")
     _need(k, "k", q.dtype)
     _need(v, "v", q.dtype, k.shape)
@@ -246,8 +261,10 @@ def sparse_attn_fwd(q, k, v, sel, *, C: int, causal: bool, scale: float = 0.0, o
         lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     if lse is not None:
         _need(lse, "lse", torch.float32, q.shape[:-1])
-    _lib.call("pisa_sparse_attn_fwd", ctypes.byref(pr.cstruct()), _p(q), _p(k), _p(v), _p(sel), _p(out), _p(lse),
-              _stream(q))
+    cfg = pr.cstruct()
+    ws = _attn_workspace(cfg, _lib.QuerySpan(0, pr.N), q.device, workspace)
+    _lib.call("pisa_sparse_attn_fwd", ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(sel), _p(out), _p(lse), _p(ws),
+              _nbytes(ws), _stream(q))
     return out, lse
 
 
@@ -286,7 +303,7 @@ def select_span(q, k, pyr, *, q0: int, C: int, K: int, causal: bool, scale: floa
 
 
 def sparse_attn_fwd_span(q, k, v, sel, *, q0: int, C: int, causal: bool, scale: float = 0.0, out=None, lse=None,
-                         want_lse: bool = True):
+                         want_lse: bool = True, workspace=None):
     """Block-sparse attention for the query rows at positions [q0, q0 + n_q):
     q [B, H_q, n_q, d] and sel [B, H_kv, n_q, K] hold those rows; k and v all
     N tokens. Returns (out [B, H_q, n_q, d], lse [B, H_q, n_q] or None)."""
@@ -302,8 +319,10 @@ def sparse_attn_fwd_span(q, k, v, sel, *, q0: int, C: int, causal: bool, scale: 
         lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     if lse is not None:
         _need(lse, "lse", torch.float32, q.shape[:-1])
-    _lib.call("pisa_sparse_attn_fwd_span", ctypes.byref(pr.cstruct()), ctypes.byref(_lib.QuerySpan(q0, n_q)), _p(q),
-              _p(k), _p(v), _p(sel), _p(out), _p(lse), _stream(q))
+    cfg, span = pr.cstruct(), _lib.QuerySpan(q0, n_q)
+    ws = _attn_workspace(cfg, span, q.device, workspace)
+    _lib.call("pisa_sparse_attn_fwd_span", ctypes.byref(cfg), ctypes.byref(span), _p(q), _p(k), _p(v), _p(sel),
+              _p(out), _p(lse), _p(ws), _nbytes(ws), _stream(q))
     return out, lse
 
 
@@ -319,7 +338,10 @@ class Prefill:
         self.cfg = pr.cstruct()
         self.pyr = torch.empty((pr.B, pr.H_kv, pr.R, pr.d), dtype=torch.float32, device=dev)
         self.sel = torch.empty((pr.B, pr.H_kv, pr.N, pr.K), dtype=torch.int32, device=dev)
-        self.ws = torch.empty(max(pr.workspace_bytes(), 16), dtype=torch.uint8, device=dev)
+        # One scratch buffer serves the selection and then the attention (the
+        # selection's scratch is dead once sel is written).
+        self.attn_ws_bytes = int(_lib.lib().pisa_attn_fwd_workspace_bytes(ctypes.byref(self.cfg)))
+        self.ws = torch.empty(max(pr.workspace_bytes(), self.attn_ws_bytes, 256), dtype=torch.uint8, device=dev)
         self.out = torch.empty((pr.B, pr.H_q, pr.N, pr.d), dtype=pr.dtype, device=dev)
         self.lse = torch.empty((pr.B, pr.H_q, pr.N), dtype=torch.float32, device=dev)
 
@@ -331,8 +353,9 @@ class Prefill:
                   _p(self.ws), self.ws.numel(), _stream(q))
 
     def attend(self, q, k, v):
+        ws = self.ws if self.attn_ws_bytes else None
         _lib.call("pisa_sparse_attn_fwd", ctypes.byref(self.cfg), _p(q), _p(k), _p(v), _p(self.sel), _p(self.out),
-                  _p(self.lse), _stream(q))
+                  _p(self.lse), _p(ws), _nbytes(ws), _stream(q))
 
     def check(self, q, k, v):
         """Raises unless q, k and v have this problem's shapes and dtype."""
@@ -366,7 +389,9 @@ class PrefillShard:
             raise ValueError(f"query span [{q0}, {q0 + n_q}) does not fit N = {pr.N}")
         self.pyr = torch.empty((pr.B, pr.H_kv, pr.R, pr.d), dtype=torch.float32, device=dev)
         self.sel = torch.empty((pr.B, pr.H_kv, n_q, pr.K), dtype=torch.int32, device=dev)
-        self.ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        self.attn_ws_bytes = int(_lib.lib().pisa_attn_fwd_span_workspace_bytes(ctypes.byref(self.cfg),
+                                                                               ctypes.byref(self.span)))
+        self.ws = torch.empty(max(nbytes, self.attn_ws_bytes, 256), dtype=torch.uint8, device=dev)
         self.out = torch.empty((pr.B, pr.H_q, n_q, pr.d), dtype=pr.dtype, device=dev)
         self.lse = torch.empty((pr.B, pr.H_q, n_q), dtype=torch.float32, device=dev)
 
@@ -378,8 +403,9 @@ class PrefillShard:
                   _p(self.sel), None, _p(self.ws), self.ws.numel(), _stream(q))
 
     def attend(self, q, k, v):
+        ws = self.ws if self.attn_ws_bytes else None
         _lib.call("pisa_sparse_attn_fwd_span", ctypes.byref(self.cfg), ctypes.byref(self.span), _p(q), _p(k), _p(v),
-                  _p(self.sel), _p(self.out), _p(self.lse), _stream(q))
+                  _p(self.sel), _p(self.out), _p(self.lse), _p(ws), _nbytes(ws), _stream(q))
 
     def check(self, q, k, v):
         """Raises unless q holds this shard's rows and k, v the whole sequence."""

@@ -205,25 +205,44 @@ pisa_status pisa_select_exact(const pisa_config* cfg, const void* q, const void*
   return from_cuda(launch_exact_rows(a, q, k, sel, as_stream(stream)));
 }
 
+size_t pisa_attn_fwd_span_workspace_bytes(const pisa_config* cfg, const pisa_query_span* span) {
+  if (check_cfg(cfg) != PISA_OK) return 0;
+  PrefillArgs a = args_of(cfg);
+  if (apply_span(span, cfg->N, &a) != PISA_OK) return 0;
+  return attn_bucket_workspace_bytes(a);
+}
+
+size_t pisa_attn_fwd_workspace_bytes(const pisa_config* cfg) {
+  if (check_cfg(cfg) != PISA_OK) return 0;
+  const pisa_query_span all{0, cfg->N};
+  return pisa_attn_fwd_span_workspace_bytes(cfg, &all);
+}
+
 pisa_status pisa_sparse_attn_fwd_span(const pisa_config* cfg, const pisa_query_span* span, const void* q,
                                       const void* k, const void* v, const int32_t* sel, void* out, float* lse,
-                                      void* stream) {
+                                      void* ws, size_t ws_bytes, void* stream) {
   pisa_status s = check_cfg(cfg);
   if (s != PISA_OK) return s;
   if (!q || !k || !v || !sel || !out) return PISA_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return PISA_ERR_INVALID_ARGUMENT;
   PrefillArgs a = args_of(cfg);
   if ((s = apply_span(span, cfg->N, &a)) != PISA_OK) return s;
+  if (ws && attn_bucket_supported(a)) {
+    if (ws_bytes < attn_bucket_workspace_bytes(a) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+      return PISA_ERR_WORKSPACE;
+    return from_cuda(launch_attn_bucket(a, q, k, v, sel, out, lse, ws, as_stream(stream)));
+  }
   if (cfg->dtype == PISA_DTYPE_BF16) return from_cuda(launch_attn_mma(a, q, k, v, sel, out, lse, as_stream(stream)));
   return from_cuda(launch_attn_rows(a, q, k, v, sel, out, lse, as_stream(stream)));
 }
 
 pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
-                                 const int32_t* sel, void* out, float* lse, void* stream) {
+                                 const int32_t* sel, void* out, float* lse, void* ws, size_t ws_bytes,
+                                 void* stream) {
   pisa_status s = check_cfg(cfg);
   if (s != PISA_OK) return s;
   const pisa_query_span all{0, cfg->N};
-  return pisa_sparse_attn_fwd_span(cfg, &all, q, k, v, sel, out, lse, stream);
+  return pisa_sparse_attn_fwd_span(cfg, &all, q, k, v, sel, out, lse, ws, ws_bytes, stream);
 }
 
 size_t pisa_attn_bwd_workspace_bytes(const pisa_config* cfg) {

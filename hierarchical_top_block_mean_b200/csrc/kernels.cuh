@@ -34,6 +34,12 @@ cudaError_t launch_flat_rows(const PrefillArgs& a, const void* q, const float* p
 // ---- tensor-core attention (bf16)
 cudaError_t launch_attn_mma(const PrefillArgs& a, const void* q, const void* k, const void* v, const int32_t* sel,
                             void* out, float* lse, cudaStream_t st);
+// Attention by leaf bucket (tcgen05; bf16, d = 128, C = 64, G_Q in {4, 8}):
+// partial softmax states per (query, block) pair in ws, then a merge.
+bool attn_bucket_supported(const PrefillArgs& a);
+size_t attn_bucket_workspace_bytes(const PrefillArgs& a);
+cudaError_t launch_attn_bucket(const PrefillArgs& a, const void* q, const void* k, const void* v, const int32_t* sel,
+                               void* out, float* lse, void* ws, cudaStream_t st);
 
 cudaError_t launch_flat_mma(const PrefillArgs& a, const void* q, const float* pyr, int64_t R, int32_t* sel,
                             cudaStream_t st);

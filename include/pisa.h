@@ -193,12 +193,28 @@ pisa_status pisa_select_exact(const pisa_config* cfg, const void* q, const void*
  *   o_t = sum_{j in T_t} exp(scale q_t.k_j) v_j / sum_{j in T_t} exp(scale q_t.k_j)
  * over the raw keys of the selected leaf blocks T_t (shared by the query heads
  * of a GQA group; keys > t excluded when causal). Negative sel entries are
- * padding; every row must select at least one usable block.
+ * padding; the blocks of a row must be distinct, and every row must select at
+ * least one usable block.
  *   sel : [B, H_kv, N, K] int32;  out : [B, H_q, N, d] in cfg->dtype;
  *   lse : NULL or [B, H_q, N] fp32, natural-log softmax denominator.
+ *   ws  : NULL, or device scratch of at least pisa_attn_fwd_workspace_bytes(cfg)
+ *         bytes, 256-byte aligned, caller-owned, contents on entry ignored.
+ * With a workspace, bf16 problems with d = 128, C = 64 and G_Q in {4, 8} run
+ * by leaf bucket: the selection is inverted per (kv head, query window, leaf),
+ * each selected block's K and V are loaded once per tile of the queries that
+ * chose it, each (query, block) pair leaves a partial softmax state
+ * (max, sum, normalised output; about G_Q * 264 bytes) in the workspace, and
+ * a merge pass combines every row's K partials in slot order. The workspace
+ * is large (K partials per query row: about 18 GB at N = 262144, H_kv = 2,
+ * G_Q = 8, K = 16). With ws = NULL (or for other shapes) every row streams
+ * its own blocks, using no scratch. A non-NULL ws smaller than the size
+ * returns PISA_ERR_WORKSPACE before anything is enqueued. Both routes give
+ * the same results within the attention tolerance; each is deterministic.
  */
+size_t pisa_attn_fwd_workspace_bytes(const pisa_config* cfg);
 pisa_status pisa_sparse_attn_fwd(const pisa_config* cfg, const void* q, const void* k, const void* v,
-                                 const int32_t* sel, void* out, float* lse, void* stream);
+                                 const int32_t* sel, void* out, float* lse, void* ws, size_t ws_bytes,
+                                 void* stream);
 
 /*
  * Size of the device array pisa_select_noalloc uses as its scratch: 64 MiB,
@@ -285,9 +301,12 @@ size_t pisa_select_span_workspace_bytes(const pisa_config* cfg, const pisa_query
 pisa_status pisa_select_span(const pisa_config* cfg, const pisa_query_span* span, const void* q, const void* k,
                              const float* pyr, int32_t* sel, float* sel_score, void* ws, size_t ws_bytes,
                              void* stream);
+/* Scratch bytes of the bucketed attention for a shard (0 when that route
+ * does not apply to cfg, or for an invalid span). */
+size_t pisa_attn_fwd_span_workspace_bytes(const pisa_config* cfg, const pisa_query_span* span);
 pisa_status pisa_sparse_attn_fwd_span(const pisa_config* cfg, const pisa_query_span* span, const void* q,
                                       const void* k, const void* v, const int32_t* sel, void* out, float* lse,
-                                      void* stream);
+                                      void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- decode
  * §Kernels, decoding: the mean pyramid is cached; per new token only the

@@ -40,7 +40,7 @@ int main(void) {
         "span past N rejected");
   check(pisa_select(&cfg, p, p, p, p, NULL, p, whole - 1, NULL) == PISA_ERR_WORKSPACE, "small workspace rejected");
   cfg.K = 17;
-  check(pisa_sparse_attn_fwd(&cfg, p, p, p, p, p, NULL, NULL) == PISA_ERR_UNSUPPORTED, "K = 17 unsupported");
+  check(pisa_sparse_attn_fwd(&cfg, p, p, p, p, p, NULL, NULL, 0, NULL) == PISA_ERR_UNSUPPORTED, "K = 17 unsupported");
   check(pisa_launch_count() == before, "nothing launched");
 
   /* An empty timing window needs no device and records nothing. */

@@ -67,7 +67,7 @@ def test_invalid_configs_rejected_before_launch(kw, code):
     assert lib.pisa_build_pyramid(ctypes.byref(cfg), dummy, dummy, None) == code
     assert lib.pisa_select(ctypes.byref(cfg), dummy, dummy, dummy, dummy, None, dummy, 1 << 30, None) == code
     assert lib.pisa_select_flat(ctypes.byref(cfg), dummy, dummy, dummy, dummy, 1 << 30, None) == code
-    assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), dummy, dummy, dummy, dummy, dummy, None, None) == code
+    assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), dummy, dummy, dummy, dummy, dummy, None, None, 0, None) == code
     assert lib.pisa_select_exact(ctypes.byref(cfg), dummy, dummy, dummy, None) == code
     assert lib.pisa_sparse_attn_bwd(ctypes.byref(cfg), dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy,
                                     dummy, dummy, 1 << 30, None) == code
@@ -84,7 +84,7 @@ def test_null_and_misaligned_pointers_rejected():
     bad = ctypes.c_void_p(258)
     assert lib.pisa_build_pyramid(ctypes.byref(cfg), None, ok, None) == 1
     assert lib.pisa_build_pyramid(ctypes.byref(cfg), bad, ok, None) == 1
-    assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), ok, ok, ok, None, ok, None, None) == 1
+    assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), ok, ok, ok, None, ok, None, None, 0, None) == 1
     assert lib.pisa_select(ctypes.byref(cfg), None, ok, ok, ok, None, ok, 1 << 30, None) == 1
     assert lib.pisa_build_pyramid(None, ok, ok, None) == 1
 
@@ -146,9 +146,10 @@ def test_query_span_validation():
         assert lib.pisa_select_span(ctypes.byref(cfg), ctypes.byref(sp), ok, ok, ok, ok, None, ok, 1 << 30,
                                     None) == 1
         assert lib.pisa_sparse_attn_fwd_span(ctypes.byref(cfg), ctypes.byref(sp), ok, ok, ok, ok, ok, None,
-                                             None) == 1
+                                             None, 0, None) == 1
+        assert lib.pisa_attn_fwd_span_workspace_bytes(ctypes.byref(cfg), ctypes.byref(sp)) == 0
     assert lib.pisa_select_span(ctypes.byref(cfg), None, ok, ok, ok, ok, None, ok, 1 << 30, None) == 1
-    assert lib.pisa_sparse_attn_fwd_span(ctypes.byref(cfg), None, ok, ok, ok, ok, ok, None, None) == 1
+    assert lib.pisa_sparse_attn_fwd_span(ctypes.byref(cfg), None, ok, ok, ok, ok, ok, None, None, 0, None) == 1
     assert lib.pisa_select_span(ctypes.byref(cfg), ctypes.byref(part), ok, ok, ok, ok, None, ok, need - 1, None) == 3
     assert lib.pisa_launch_count() == before
 
@@ -188,3 +189,24 @@ def test_flat_workspace_sized_and_checked_before_launch():
     assert lib.pisa_select_flat(ctypes.byref(cfg), dummy, dummy, dummy, None, need, None) == 3
     assert lib.pisa_launch_count() == before
     assert lib.pisa_select_flat_workspace_bytes(ctypes.byref(_cfg(N=1000, d=64, C=32))) == 0
+
+
+def test_attention_workspace_sized_and_checked_before_launch():
+    # The bucketed attention (bf16, d = 128, C = 64, G_Q in {4, 8}) keeps a
+    # partial softmax state per (query, selected block, head) in the caller's
+    # workspace: at least rows * K * G_Q * (256 + 8) bytes. A shard needs
+    # scratch for its own rows only. Too small a workspace is refused before
+    # anything is enqueued; other shapes report 0 and stream rows without one.
+    lib = _lib.lib()
+    cfg = _cfg(N=1000, H_q=8, H_kv=2, d=128, C=64, K=16)
+    need = lib.pisa_attn_fwd_workspace_bytes(ctypes.byref(cfg))
+    assert need >= 2 * 1000 * 16 * 4 * 264
+    half = _lib.QuerySpan(500, 500)
+    assert 0 < lib.pisa_attn_fwd_span_workspace_bytes(ctypes.byref(cfg), ctypes.byref(half)) < need
+    before = lib.pisa_launch_count()
+    ok = ctypes.c_void_p(1024)
+    assert lib.pisa_sparse_attn_fwd(ctypes.byref(cfg), ok, ok, ok, ok, ok, None, ok, need - 1, None) == 3
+    assert lib.pisa_launch_count() == before
+    for kw in (dict(d=64, C=32), dict(H_q=2, H_kv=2, d=128, C=64), dict(d=128, C=32, H_q=8, H_kv=2),
+               dict(dtype=0, d=128, C=64, H_q=8, H_kv=2)):
+        assert lib.pisa_attn_fwd_workspace_bytes(ctypes.byref(_cfg(N=1000, **kw))) == 0
