@@ -198,6 +198,8 @@ def work_model(w):
         "flat_flops": heads * v1.sum() * 2 * w.d,
         "exact_flops": heads * v1.sum() * 2 * G * w.C * w.d,
         "final_bytes": heads * w.N * (32 * 8 + K * 4),
+        "attn_partial_bytes": heads * w.N * K * G * (128 * 2 + 8),
+        "attn_out_bytes": w.B * w.H_q * w.N * (w.d * e + 4),
         "split_bytes": heads * api.pyramid_rows(w.N, w.C) * w.d * 8,
     }.items()}
 
@@ -310,6 +312,13 @@ def kernel_rooflines(w, kern, flat_ms, exact_ms, decode, pk, pk_kind):
             hbm_unique_gbs=m["attn_unique_bytes"] / (a[0] * 1e-3) / 1e9,
             hbm_unique_frac=m["attn_unique_bytes"] / (a[0] * 1e-3) / 1e9 / hbm,
             l2_gather_gbs=attn_bytes(w) / (a[0] * 1e-3) / 1e9)
+    ab = k("attn_bucket_kernel")
+    if ab[0]:
+        add("attn_bucket_kernel", *ab, "tensor", m["attn_flops"],
+            "4 G_Q d flops per usable key of the K selected blocks; also writes the partial states",
+            partial_write_gbs=m["attn_partial_bytes"] / (ab[0] * 1e-3) / 1e9)
+    add("attn_merge_kernel", *k("attn_merge_kernel"), "hbm", m["attn_partial_bytes"] + m["attn_out_bytes"],
+        "partial states of every (query, selected block, head) read once; out and lse written")
     add("flat_mma_kernel", flat_ms, 1, "tensor", m["flat_flops"],
         "2 d flops per (query row, usable leaf) after the group sum; not part of the step")
     add("exact_umma_kernel", exact_ms, 1, "tensor", m["exact_flops"],

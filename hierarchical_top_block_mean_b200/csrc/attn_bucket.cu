@@ -29,9 +29,9 @@
 //   warps 8-11 (loads): per tile, the 128 (query, head) rows by 16-byte
 //     cp.async into a ring of kAbQStages 128-byte-swizzled stages;
 //   warp 12, one lane: per item the K and V^T tiles by bulk tensor copy
-//     (double buffered, requested as soon as a stage frees); per tile n the S
-//     MMAs, then the O MMAs of tile n - 2, so an epilogue group forms P
-//     while later S tiles are computed;
+//     (double buffered, requested as soon as a stage frees); it polls the
+//     pipeline, issuing each tile's S MMAs and, once the tile's P is in
+//     shared memory, its O MMAs, whichever is ready first;
 //   warps 0-7 (epilogue): two groups of four warps take alternate tiles (TMEM
 //     stage = tile parity); each thread owns one (query, head) row.
 // Every mbarrier wait is bounded in time; the TMEM allocation is released
@@ -394,12 +394,15 @@ __global__ void __launch_bounds__(kAbThreads, 1)
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
       // Item j of this CTA (item blockIdx.x + j gridDim.x) uses K/V stage
-      // j & 1. The O MMAs of a tile are issued two tiles after its S MMAs, so
-      // an epilogue group forms P while later S tiles are computed. The O
-      // MMAs of an item's last tile free its K/V stage; the tiles of item
-      // j + 2 are then requested at once. Before a new item waits for its K/V
-      // stage, the O MMAs of the item two back (that stage's last user) are
-      // issued, so the wait can always be met.
+      // j & 1; the O MMAs of an item's last tile free it, and the tiles of
+      // item j + 2 are requested at once. One thread issues every MMA, so it
+      // never blocks on one epilogue group while the other could use the
+      // tensor cores: it polls, issuing the oldest pending O MMAs once their
+      // P is ready, and the next tile's S MMAs once its queries, its TMEM
+      // stage and its K/V tile are (a new item first needs the O MMAs of the
+      // item two back, its stage's last user). S runs in tile order and O in
+      // tile order. With no progress for kWaitNs the loop gives up (counted
+      // as a fault), like every bounded wait.
       auto load_kv = [&](int j) {
         const int it = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
         if (it >= total) return;
@@ -416,58 +419,69 @@ __global__ void __launch_bounds__(kAbThreads, 1)
         int n, j;
         bool last;
       };
-      Pend fifo[3];
+      constexpr int kF = 4;  // S issued, O pending: at most two tiles per TMEM stage
+      Pend fifo[kF];
       int f_head = 0, f_len = 0;
-      auto issue_o = [&]() {
-        const Pend pd = fifo[f_head];
-        f_head = (f_head + 1) % 3;
-        --f_len;
-        const int s = pd.n & 1, u = pd.n >> 1, kb = pd.j & 1;
-        mbar_wait(&pfull[s], u & 1, faults);
-        tc_fence_after();
-        const uint32_t pa = smem_u32(pbuf + s * kAbPBytes), vb = smem_u32(vbuf + kb * kAbVBytes);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          umma_bf16(tmem + 256 * s + 128, sw128_desc(pa + ks * 32), sw128_desc(vb + ks * 32), kIdescO, ks > 0);
-        umma_commit(&ofull[s]);
-        if (pd.last) {
-          umma_commit(&kvempty[kb]);
-          load_kv(pd.j + 2);
-        }
-      };
       load_kv(0);
       load_kv(1);
       Stream sm = stream_begin();
       int n = 0, j = -1;
-      while (sm.item < total) {
-        const Stream cur = sm;
-        sm = stream_next(sm);
-        if (cur.tl == 0) {
-          ++j;
-          while (f_len > 0 && fifo[f_head].j <= j - 2) issue_o();
-          mbar_wait(&kvfull[j & 1], (j >> 1) & 1, faults);
-        }
-        const int kb = j & 1;
-        const int s = n & 1, u = n >> 1;
-        const int qs = n % kAbQStages;
-        mbar_wait(&qfull[qs], (n / kAbQStages) & 1, faults);
-        mbar_wait(&sfree[s], (u & 1) ^ 1, faults);  // the group has read S of tile n - 2
-        tc_fence_after();
-        const uint32_t qa = smem_u32(qbuf + qs * kAbQBytes), ka = smem_u32(kbuf + kb * kAbKBytes);
+      uint64_t t_prog = global_ns();
+      while (sm.item < total || f_len > 0) {
+        bool prog = false;
+        if (f_len > 0) {
+          const Pend pd = fifo[f_head];
+          const int s = pd.n & 1, u = pd.n >> 1, kb = pd.j & 1;
+          if (mbar_test(&pfull[s], u & 1)) {
+            tc_fence_after();
+            const uint32_t pa = smem_u32(pbuf + s * kAbPBytes), vb = smem_u32(vbuf + kb * kAbVBytes);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t qo = (ks >> 2) * (kAbQBytes / 2) + (ks & 3) * 32;
-          const uint32_t ko = (ks >> 2) * (kAbKBytes / 2) + (ks & 3) * 32;
-          umma_bf16(tmem + 256 * s, sw128_desc(qa + qo), sw128_desc(ka + ko), kIdescS, ks > 0);
+            for (int ks = 0; ks < 4; ++ks)
+              umma_bf16(tmem + 256 * s + 128, sw128_desc(pa + ks * 32), sw128_desc(vb + ks * 32), kIdescO, ks > 0);
+            umma_commit(&ofull[s]);
+            f_head = (f_head + 1) % kF;
+            --f_len;
+            if (pd.last) {
+              umma_commit(&kvempty[kb]);
+              load_kv(pd.j + 2);
+            }
+            prog = true;
+          }
         }
-        umma_commit(&qempty[qs]);
-        umma_commit(&sfull[s]);
-        fifo[(f_head + f_len) % 3] = Pend{n, j, cur.tl + 1 == cur.ntiles};
-        ++f_len;
-        if (f_len == 3) issue_o();  // the O MMAs of tile n - 2
-        ++n;
+        if (sm.item < total && f_len < kF) {
+          const bool first = sm.tl == 0;
+          const int jn = first ? j + 1 : j;
+          const int s = n & 1, u = n >> 1, qs = n % kAbQStages;
+          bool ready = !(first && f_len > 0 && fifo[f_head].j <= jn - 2);
+          ready = ready && (!first || mbar_test(&kvfull[jn & 1], (jn >> 1) & 1));
+          ready = ready && mbar_test(&qfull[qs], (n / kAbQStages) & 1);
+          ready = ready && mbar_test(&sfree[s], (u & 1) ^ 1);  // the group has read S of tile n - 2
+          if (ready) {
+            j = jn;
+            tc_fence_after();
+            const uint32_t qa = smem_u32(qbuf + qs * kAbQBytes), ka = smem_u32(kbuf + (j & 1) * kAbKBytes);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint32_t qo = (ks >> 2) * (kAbQBytes / 2) + (ks & 3) * 32;
+              const uint32_t ko = (ks >> 2) * (kAbKBytes / 2) + (ks & 3) * 32;
+              umma_bf16(tmem + 256 * s, sw128_desc(qa + qo), sw128_desc(ka + ko), kIdescS, ks > 0);
+            }
+            umma_commit(&qempty[qs]);
+            umma_commit(&sfull[s]);
+            fifo[(f_head + f_len) % kF] = Pend{n, j, sm.tl + 1 == sm.ntiles};
+            ++f_len;
+            sm = stream_next(sm);
+            ++n;
+            prog = true;
+          }
+        }
+        if (prog) {
+          t_prog = global_ns();
+        } else if (global_ns() - t_prog > kWaitNs) {
+          if (faults) atomicAdd(faults, 1ull);
+          break;
+        }
       }
-      while (f_len > 0) issue_o();
     }
   } else {
     // ---------------------------------------------------------- epilogue

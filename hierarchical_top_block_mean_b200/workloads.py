@@ -106,6 +106,10 @@ PREFILL = {
     # and parity case for the G_Q = 8 kernels that still exceeds L2 (q: 268 MB).
     "needle_64k_g8": Prefill("needle_64k_g8", B=1, N=65536, H_q=16, H_kv=2, d=128, C=64, K=16, causal=True,
                              dtype="bf16", structure="needle", n_needles=64, seed=4500),
+    # Half that again: q (134 MB) still exceeds L2, and the whole step fits in
+    # about 2.5 GB of device memory, the size for single-kernel profiler captures.
+    "needle_32k_g8": Prefill("needle_32k_g8", B=1, N=32768, H_q=16, H_kv=2, d=128, C=64, K=16, causal=True,
+                             dtype="bf16", structure="needle", n_needles=32, seed=4600),
 }
 
 DECODE = {
