@@ -26,14 +26,16 @@
 // attn_bucket_kernel (partials), attn_merge_kernel.
 //
 // attn_bucket_kernel is persistent (one CTA per SM) and warp-specialised:
-//   warps 8-11 (loads): per tile, the 128 (query, head) rows by 16-byte
+//   warps 12-13 (loads): per tile, the 128 (query, head) rows by 16-byte
 //     cp.async into a ring of kAbQStages 128-byte-swizzled stages;
-//   warp 12, one lane: per item the K and V^T tiles by bulk tensor copy
+//   warp 14, one lane: per item the K and V^T tiles by bulk tensor copy
 //     (double buffered, requested as soon as a stage frees); it polls the
 //     pipeline, issuing each tile's S MMAs and, once the tile's P is in
 //     shared memory, its O MMAs, whichever is ready first;
-//   warps 0-7 (epilogue): two groups of four warps take alternate tiles (TMEM
-//     stage = tile parity); each thread owns one (query, head) row.
+//   warps 0-11 (epilogue): three groups of four warps take tiles in turn
+//     (group = TMEM stage = tile index mod 3); each thread owns one (query,
+//     head) row. A stage's S columns are overwritten by its O once the group
+//     has formed P, and the stage takes a new tile once O has been read.
 // Every mbarrier wait is bounded in time; the TMEM allocation is released
 // before exit.
 #include <algorithm>
@@ -48,19 +50,22 @@ namespace pisa {
 namespace {
 
 constexpr int kAbItemPairs = 64;
-constexpr int kAbEpiWarps = 8;
-constexpr int kAbLoadWarps = 4;
+constexpr int kAbGroups = 3;                    // epilogue groups = TMEM stages
+constexpr int kAbEpiWarps = 4 * kAbGroups;
+constexpr int kAbLoadWarps = 2;
 constexpr int kAbMmaWarp = kAbEpiWarps + kAbLoadWarps;
 constexpr int kAbThreads = 32 * (kAbMmaWarp + 1);
 constexpr int kAbLoaders = 32 * kAbLoadWarps;
-constexpr int kAbQStages = 4;
-constexpr int kAbLag = 2;                       // a query stage is published kAbLag tiles after it is filled
+constexpr int kAbQStages = 3;
+constexpr int kAbLag = 1;                       // a query stage is published kAbLag tiles after it is filled
 constexpr int kAbQBytes = 128 * 128 * 2;        // 128 rows x 128 bf16 (two 64-column halves)
 constexpr int kAbKBytes = 64 * 128 * 2;         // 64 keys x 128 d (two halves)
 constexpr int kAbVBytes = 128 * 64 * 2;         // 128 d x 64 keys (one box)
 constexpr int kAbPBytes = 128 * 64 * 2;         // 128 rows x 64 keys
-constexpr int kAbSmem = 1024 + 2 * (kAbKBytes + kAbVBytes) + kAbQStages * kAbQBytes + 2 * kAbPBytes;
-constexpr uint32_t kAbTmemCols = 512;            // stage s: S at 256 s, O at 256 s + 128
+constexpr int kAbSmem = 1024 + 2 * (kAbKBytes + kAbVBytes) + kAbQStages * kAbQBytes + kAbGroups * kAbPBytes;
+// Stage s occupies TMEM columns [128 s, 128 s + 128): S in its first 64, then
+// O over all 128 once S has been read.
+constexpr uint32_t kAbTmemCols = 512;
 // Instruction descriptors (kind::f16, bf16 A and B, fp32 D, both K-major).
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescO = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -266,23 +271,25 @@ __global__ void __launch_bounds__(kAbThreads, 1)
   constexpr int TQ = 128 / G;  // queries per tile
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ uint64_t kvfull[2], kvempty[2], qfull[kAbQStages], qempty[kAbQStages];
-  __shared__ uint64_t sfull[2], pfull[2], ofull[2], sfree[2];
+  __shared__ uint64_t sfull[kAbGroups], pfull[kAbGroups], ofull[kAbGroups], tfree[kAbGroups];
   __shared__ uint32_t tmem_base_sh;
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* kbuf = smem;                                   // [2][kAbKBytes]
   unsigned char* vbuf = kbuf + 2 * kAbKBytes;                   // [2][kAbVBytes]
   unsigned char* qbuf = vbuf + 2 * kAbVBytes;                   // [kAbQStages][kAbQBytes]
-  unsigned char* pbuf = qbuf + kAbQStages * kAbQBytes;          // [2][kAbPBytes]
+  unsigned char* pbuf = qbuf + kAbQStages * kAbQBytes;          // [kAbGroups][kAbPBytes]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kvfull[i], 1);
       mbar_init(&kvempty[i], 1);
+    }
+    for (int i = 0; i < kAbGroups; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 4);
       mbar_init(&ofull[i], 1);
-      mbar_init(&sfree[i], 4);
+      mbar_init(&tfree[i], 4);
     }
     for (int i = 0; i < kAbQStages; ++i) {
       mbar_init(&qfull[i], kAbLoaders);
@@ -338,7 +345,6 @@ __global__ void __launch_bounds__(kAbThreads, 1)
     // r is head r % G of the tile's query r / G.
     const int lw = warp - kAbEpiWarps;
     const int jcol = lane & 15;
-    const int slot = 2 * lw + (lane >> 4);
     const int64_t head_stride = static_cast<int64_t>(a.Nq) * 128;
     int nq = 0;
     int pend[kAbLag + 1] = {}, np_head = 0, npend = 0;
@@ -361,7 +367,10 @@ __global__ void __launch_bounds__(kAbThreads, 1)
       mbar_wait(&qempty[qs], ((nq / kAbQStages) & 1) ^ 1, faults);
       const uint32_t qd = smem_u32(qbuf + qs * kAbQBytes) + (jcol >> 3) * (kAbQBytes / 2);
 #pragma unroll
+      for (int sl = 0; sl < 8 / (2 * kAbLoadWarps); ++sl)
+#pragma unroll
       for (int m = 0; m < 16; ++m) {
+        const int slot = 2 * lw + (lane >> 4) + 2 * kAbLoadWarps * sl;
         const int r = slot + 8 * m;
         const int qi = r / G, hd = r % G;
         const uint32_t wq = __shfl_sync(kFull, twv, qi);
@@ -419,7 +428,7 @@ __global__ void __launch_bounds__(kAbThreads, 1)
         int n, j;
         bool last;
       };
-      constexpr int kF = 4;  // S issued, O pending: at most two tiles per TMEM stage
+      constexpr int kF = kAbGroups;  // S issued, O pending: at most one tile per TMEM stage
       Pend fifo[kF];
       int f_head = 0, f_len = 0;
       load_kv(0);
@@ -431,13 +440,13 @@ __global__ void __launch_bounds__(kAbThreads, 1)
         bool prog = false;
         if (f_len > 0) {
           const Pend pd = fifo[f_head];
-          const int s = pd.n & 1, u = pd.n >> 1, kb = pd.j & 1;
+          const int s = pd.n % kAbGroups, u = pd.n / kAbGroups, kb = pd.j & 1;
           if (mbar_test(&pfull[s], u & 1)) {
             tc_fence_after();
             const uint32_t pa = smem_u32(pbuf + s * kAbPBytes), vb = smem_u32(vbuf + kb * kAbVBytes);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-              umma_bf16(tmem + 256 * s + 128, sw128_desc(pa + ks * 32), sw128_desc(vb + ks * 32), kIdescO, ks > 0);
+              umma_bf16(tmem + 128 * s, sw128_desc(pa + ks * 32), sw128_desc(vb + ks * 32), kIdescO, ks > 0);
             umma_commit(&ofull[s]);
             f_head = (f_head + 1) % kF;
             --f_len;
@@ -451,11 +460,11 @@ __global__ void __launch_bounds__(kAbThreads, 1)
         if (sm.item < total && f_len < kF) {
           const bool first = sm.tl == 0;
           const int jn = first ? j + 1 : j;
-          const int s = n & 1, u = n >> 1, qs = n % kAbQStages;
+          const int s = n % kAbGroups, u = n / kAbGroups, qs = n % kAbQStages;
           bool ready = !(first && f_len > 0 && fifo[f_head].j <= jn - 2);
           ready = ready && (!first || mbar_test(&kvfull[jn & 1], (jn >> 1) & 1));
           ready = ready && mbar_test(&qfull[qs], (n / kAbQStages) & 1);
-          ready = ready && mbar_test(&sfree[s], (u & 1) ^ 1);  // the group has read S of tile n - 2
+          ready = ready && mbar_test(&tfree[s], (u & 1) ^ 1);  // the group has read O of tile n - kAbGroups
           if (ready) {
             j = jn;
             tc_fence_after();
@@ -464,7 +473,7 @@ __global__ void __launch_bounds__(kAbThreads, 1)
             for (int ks = 0; ks < 8; ++ks) {
               const uint32_t qo = (ks >> 2) * (kAbQBytes / 2) + (ks & 3) * 32;
               const uint32_t ko = (ks >> 2) * (kAbKBytes / 2) + (ks & 3) * 32;
-              umma_bf16(tmem + 256 * s, sw128_desc(qa + qo), sw128_desc(ka + ko), kIdescS, ks > 0);
+              umma_bf16(tmem + 128 * s, sw128_desc(qa + qo), sw128_desc(ka + ko), kIdescS, ks > 0);
             }
             umma_commit(&qempty[qs]);
             umma_commit(&sfull[s]);
@@ -486,7 +495,7 @@ __global__ void __launch_bounds__(kAbThreads, 1)
   } else {
     // ---------------------------------------------------------- epilogue
     const float sl2 = a.scale * 1.4426950408889634f;
-    const int grp = warp >> 2, qtr = warp & 3;
+    const int grp = warp >> 2, qtr = warp & 3;  // group grp takes tiles grp, grp + kAbGroups, ...
     const int r = 32 * qtr + lane;  // TMEM lane = tile row = query r / G, head r % G
     const int hd = r % G;
     auto row_word = [&](const Stream& st) -> uint32_t {
@@ -494,21 +503,23 @@ __global__ void __launch_bounds__(kAbThreads, 1)
       const int p = st.inf.y + st.tl * TQ + r / G;
       return p < st.inf.z ? ws.pairs[p] : 0xffffffffu;
     };
+    auto advance = [&](Stream st) {
+#pragma unroll
+      for (int i = 0; i < kAbGroups; ++i) st = stream_next(st);
+      return st;
+    };
     Stream sm = stream_begin();
     int n = 0;
-    if (grp == 1) {
-      sm = stream_next(sm);
-      n = 1;
-    }
+    for (; n < grp; ++n) sm = stream_next(sm);
     uint32_t w_next = row_word(sm);
     while (sm.item < total) {
       const int4 inf = sm.inf;
       const uint32_t w = w_next;
       const int ncur = n;
-      sm = stream_next(stream_next(sm));
-      n += 2;
+      sm = advance(sm);
+      n += kAbGroups;
       w_next = row_word(sm);
-      const int s = ncur & 1, u = ncur >> 1;
+      const int s = ncur % kAbGroups, u = ncur / kAbGroups;
       const bool ok = w != 0xffffffffu;
       const int64_t i_row = ok ? static_cast<int64_t>(w >> 5) : 0;
       const int64_t key0 = static_cast<int64_t>(inf.w) * 64;
@@ -518,11 +529,8 @@ __global__ void __launch_bounds__(kAbThreads, 1)
       __syncwarp();
       tc_fence_after();
       uint32_t v[64];
-      tmem_ld_cols<64>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + 256 * s, v);
+      tmem_ld_cols<64>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + 128 * s, v);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sfree[s]);  // S of this stage may be overwritten
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (nv >= 64) {
 #pragma unroll
@@ -565,7 +573,7 @@ __global__ void __launch_bounds__(kAbThreads, 1)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t o[64];
-        tmem_ld_cols<64>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + 256 * s + 128 + 64 * c, o);
+        tmem_ld_cols<64>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + 128 * s + 64 * c, o);
         tmem_ld_wait();
         if (ok) {
 #pragma unroll
@@ -585,6 +593,7 @@ __global__ void __launch_bounds__(kAbThreads, 1)
       if (ok) ws.part_ml[pair * G + hd] = make_float2(nv > 0 ? mx * a.scale : -INFINITY, l);
       tc_fence_before();
       __syncwarp();
+      if (lane == 0) mbar_arrive(&tfree[s]);  // the stage may take the next tile's S
     }
   }
   tc_fence_before();
