@@ -319,8 +319,9 @@ def kernel_rooflines(w, kern, flat_ms, exact_ms, decode, pk, pk_kind):
             partial_write_gbs=m["attn_partial_bytes"] / (ab[0] * 1e-3) / 1e9)
     add("attn_merge_kernel", *k("attn_merge_kernel"), "hbm", m["attn_partial_bytes"] + m["attn_out_bytes"],
         "partial states of every (query, selected block, head) read once; out and lse written")
-    add("flat_mma_kernel", flat_ms, 1, "tensor", m["flat_flops"],
-        "2 d flops per (query row, usable leaf) after the group sum; not part of the step")
+    add("flat_selector", flat_ms, 1, "tensor", m["flat_flops"],
+        "one pisa_select_flat call (flat_prep_kernel + flat_umma_kernel at d = 128); 2 d flops per "
+        "(query row, usable leaf) after the group sum; not part of the step")
     add("exact_umma_kernel", exact_ms, 1, "tensor", m["exact_flops"],
         "2 G_Q C d flops per (query row, usable leaf); not part of the step")
     if decode:

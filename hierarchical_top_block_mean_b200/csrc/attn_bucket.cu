@@ -13,10 +13,10 @@
 //   P = exp(scale S - m) per row over its usable keys, m the row maximum,
 //       l = sum of P (bf16 P written to shared memory as the next A operand)
 //   O [128 rows x 128 d]    = P V                    (B = V^T, K-major)
-// and each pair writes its partial (m, l, O / l) per head; l sums the fp32 P
-// (the O MMA takes P rounded to bf16). attn_merge_kernel
-// then combines the K partials of every (query, head) in slot order:
-//   M = max m_k, L = sum l_k e^{m_k - M}, o = sum (l_k e^{m_k - M} / L) O_k/l_k,
+// and each pair writes its partial (m, l, O) per head, O unnormalised; l sums
+// the fp32 P (the O MMA takes P rounded to bf16). attn_merge_kernel then
+// combines the K partials of every (query, head) in slot order:
+//   M = max m_k, L = sum l_k e^{m_k - M}, o = sum (e^{m_k - M} / L) O_k,
 //   lse = M + log L.
 // The result of a pair does not depend on which other pairs share its tile,
 // and the merge order is fixed, so the output is reproducible bit for bit.
@@ -26,14 +26,14 @@
 // attn_bucket_kernel (partials), attn_merge_kernel.
 //
 // attn_bucket_kernel is persistent (one CTA per SM) and warp-specialised:
-//   warps 12-13 (loads): per tile, the 128 (query, head) rows by 16-byte
+//   warps 16-17 (loads): per tile, the 128 (query, head) rows by 16-byte
 //     cp.async into a ring of kAbQStages 128-byte-swizzled stages;
-//   warp 14, one lane: per item the K and V^T tiles by bulk tensor copy
+//   warp 18, one lane: per item the K and V^T tiles by bulk tensor copy
 //     (double buffered, requested as soon as a stage frees); it polls the
 //     pipeline, issuing each tile's S MMAs and, once the tile's P is in
 //     shared memory, its O MMAs, whichever is ready first;
-//   warps 0-11 (epilogue): three groups of four warps take tiles in turn
-//     (group = TMEM stage = tile index mod 3); each thread owns one (query,
+//   warps 0-15 (epilogue): four groups of four warps take tiles in turn
+//     (group = TMEM stage = tile index mod 4); each thread owns one (query,
 //     head) row. A stage's S columns are overwritten by its O once the group
 //     has formed P, and the stage takes a new tile once O has been read.
 // Every mbarrier wait is bounded in time; the TMEM allocation is released
@@ -50,7 +50,7 @@ namespace pisa {
 namespace {
 
 constexpr int kAbItemPairs = 64;
-constexpr int kAbGroups = 3;                    // epilogue groups = TMEM stages
+constexpr int kAbGroups = 4;                    // epilogue groups = TMEM stages
 constexpr int kAbEpiWarps = 4 * kAbGroups;
 constexpr int kAbLoadWarps = 2;
 constexpr int kAbMmaWarp = kAbEpiWarps + kAbLoadWarps;
@@ -78,7 +78,7 @@ struct AbWs {
   uint32_t* pairs;      // [rows K] (query row << 5 | slot), grouped by bucket
   int4* item_info;      // [items] {bh, first pair, end pair, leaf}
   bf16* vt;             // [B H_kv][128][Np] V transposed, keys padded to Np
-  bf16* part_o;         // [rows K][16 chunks][G][8] O_k / l_k per (pair, head)
+  bf16* part_o;         // [rows K][16 chunks][G][8] O_k (unnormalised) per (pair, head)
   float2* part_ml;      // [rows K G] (m_k, l_k)
   int win_shift, nwin;
   int64_t Np;
@@ -528,35 +528,49 @@ __global__ void __launch_bounds__(kAbThreads, 1)
       mbar_wait(&sfull[s], u & 1, faults);
       __syncwarp();
       tc_fence_after();
-      uint32_t v[64];
-      tmem_ld_cols<64>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + 128 * s, v);
-      tmem_ld_wait();
+      // S is read from TMEM twice, 32 columns at a time (maximum, then
+      // exponentials), to keep the epilogue within the registers that four
+      // groups of warps can hold.
+      const uint32_t srow = tmem + (static_cast<uint32_t>(32 * qtr) << 16) + 128 * s;
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (nv >= 64) {
 #pragma unroll
-        for (int jj = 0; jj < 64; ++jj) m4[jj & 3] = fmaxf(m4[jj & 3], __uint_as_float(v[jj]));
-      } else {
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t v[32];
+        tmem_ld32(srow + 32 * h2, v);
+        tmem_ld_wait();
+        if (nv >= 32 * h2 + 32) {
 #pragma unroll
-        for (int jj = 0; jj < 64; ++jj)
-          if (jj < nv) m4[jj & 3] = fmaxf(m4[jj & 3], __uint_as_float(v[jj]));
+          for (int jj = 0; jj < 32; ++jj) m4[jj & 3] = fmaxf(m4[jj & 3], __uint_as_float(v[jj]));
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (32 * h2 + jj < nv) m4[jj & 3] = fmaxf(m4[jj & 3], __uint_as_float(v[jj]));
+        }
       }
       const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       const float mxs = nv > 0 ? mx * sl2 : 0.f;
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
       unsigned char* prow = pbuf + s * kAbPBytes + r * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t pk[4];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t v[32];
+        tmem_ld32(srow + 32 * h2, v);
+        tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j0 = 8 * c + 2 * e;
-          const float p0 = j0 < nv ? ex2_approx(fmaf(__uint_as_float(v[j0]), sl2, -mxs)) : 0.f;
-          const float p1 = j0 + 1 < nv ? ex2_approx(fmaf(__uint_as_float(v[j0 + 1]), sl2, -mxs)) : 0.f;
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
-          l4[e] += p0 + p1;
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int jl = 8 * c + 2 * e, j0 = 32 * h2 + jl;
+            const float p0 = j0 < nv ? ex2_approx(fmaf(__uint_as_float(v[jl]), sl2, -mxs)) : 0.f;
+            const float p1 = j0 + 1 < nv ? ex2_approx(fmaf(__uint_as_float(v[jl + 1]), sl2, -mxs)) : 0.f;
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&pb);
+            l4[e] += p0 + p1;
+          }
+          const int cc = 4 * h2 + c;
+          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
       fence_proxy_async();  // the O MMA reads P through the async proxy
@@ -566,26 +580,25 @@ __global__ void __launch_bounds__(kAbThreads, 1)
       __syncwarp();
       tc_fence_after();
       // Partial layout per pair: [16 column chunks of 8][G heads][8] bf16, so
-      // the 8 heads of a pair write each chunk as one 128-byte line.
+      // the G heads of a pair write each chunk as one contiguous piece. O is
+      // stored unnormalised (P relative to the row maximum); (m, l) go beside it.
       const int64_t pair = (static_cast<int64_t>(inf.x) * a.Nq + i_row) * a.K + (ok ? (w & 31) : 0);
-      const float inv = l > 0.f ? 1.f / l : 0.f;
       bf16* dst = ws.part_o + pair * (G * 128) + hd * 8;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t o[64];
-        tmem_ld_cols<64>(tmem + (static_cast<uint32_t>(32 * qtr) << 16) + 128 * s + 64 * c, o);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(srow + 32 * c, o);
         tmem_ld_wait();
         if (ok) {
 #pragma unroll
-          for (int e = 0; e < 64; e += 8) {
+          for (int e = 0; e < 32; e += 8) {
             uint32_t pk[4];
 #pragma unroll
             for (int f = 0; f < 4; ++f) {
-              const __nv_bfloat162 ob =
-                  __floats2bfloat162_rn(__uint_as_float(o[e + 2 * f]) * inv, __uint_as_float(o[e + 2 * f + 1]) * inv);
+              const __nv_bfloat162 ob = __floats2bfloat162_rn(__uint_as_float(o[e + 2 * f]), __uint_as_float(o[e + 2 * f + 1]));
               pk[f] = *reinterpret_cast<const uint32_t*>(&ob);
             }
-            const int chunk = (64 * c + e) / 8;
+            const int chunk = (32 * c + e) / 8;
             *reinterpret_cast<uint4*>(dst + chunk * (G * 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
@@ -642,8 +655,8 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const int32_t* __restri
     float M = m[i];
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-    const float e = l[i] > 0.f ? l[i] * expf(m[i] - M) : 0.f;
-    float L = e;
+    const float e = l[i] > 0.f ? expf(m[i] - M) : 0.f;  // scale of slot k's P relative to the row maximum
+    float L = e * l[i];
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) L += __shfl_xor_sync(kFull, L, o);
     wt[i] = L > 0.f ? e / L : 0.f;

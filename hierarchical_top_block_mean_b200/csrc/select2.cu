@@ -77,11 +77,6 @@ size_t carve(const PrefillArgs& a, char* base, Ws* w) {
   return o;
 }
 
-__device__ inline bool usable(int64_t n, int C, int l, int64_t i, int64_t t, bool causal) {
-  if (i < 0 || i >= level_size(n, C, l)) return false;
-  return !causal || i * level_span(C, l) <= t;
-}
-
 // Pyramid rows (fp32) -> interleaved bf16 hi/lo chunks, so that the router
 // reads ready MMA operands: chunk c of a row holds hi(x[4c..4c+3]) then
 // lo(x[4c..4c+3]), with x - hi - lo below 2^-16 |x|.
@@ -143,8 +138,12 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
       qb[ks][0] = gid < G ? u.x : 0u;
       qb[ks][1] = gid < G ? u.y : 0u;
     }
+    // Usable blocks of a level are exactly the first valid_count of them, so
+    // one count per level replaces a per-candidate test.
+    int vc = static_cast<int>(valid_count(n, C, l, t, causal));
     for (; l >= 2; --l) {
-      const int nc = warp_compact(cand, cand >= 0 && usable(n, C, l, cand, t, causal), tmp[warp]);
+      const int vcc = static_cast<int>(valid_count(n, C, l - 1, t, causal));  // usable children level
+      const int nc = warp_compact(cand, cand >= 0 && cand < vc, tmp[warp]);
       int nk = nc;
       if (nc > K) {
         // M-tile m holds candidates 8m .. 8m+7: row gid = first child, row gid + 8 = second.
@@ -155,7 +154,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
           const int c = __shfl_sync(kFull, cand, 8 * m + gid);
           const bool have = 8 * m + gid < nc;
           const int64_t r0 = have ? 2 * static_cast<int64_t>(c) : 0;
-          const bool has1 = have && usable(n, C, l - 1, r0 + 1, t, causal);
+          const bool has1 = have && r0 + 1 < vcc;
           const uint4* p0 = PL + (off[l - 1] + r0) * (D / 4) + tig;
           const uint4* p1 = PL + (off[l - 1] + (has1 ? r0 + 1 : r0)) * (D / 4) + tig;
           uint4 x0[D / 16], x1[D / 16];
@@ -204,10 +203,11 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
       }
       const int parent = __shfl_sync(kFull, cand, lane >> 1);
       cand = (lane >> 1) < nk ? 2 * parent + (lane & 1) : -1;
+      vc = vcc;
     }
   }
   // Leaf-level candidates.
-  const int nc = warp_compact(cand, cand >= 0 && usable(n, C, 1, cand, t, causal), tmp[warp]);
+  const int nc = warp_compact(cand, cand >= 0 && cand < static_cast<int>(valid_count(n, C, 1, t, causal)), tmp[warp]);
   if (nc <= K) {
     int idx = lane < nc ? cand : INT_MAX;
     warp_sort_asc(idx);
