@@ -57,7 +57,6 @@ constexpr int kAbMmaWarp = kAbEpiWarps + kAbLoadWarps;
 constexpr int kAbThreads = 32 * (kAbMmaWarp + 1);
 constexpr int kAbLoaders = 32 * kAbLoadWarps;
 constexpr int kAbQStages = 3;
-constexpr int kAbLag = 1;                       // a query stage is published kAbLag tiles after it is filled
 constexpr int kAbQBytes = 128 * 128 * 2;        // 128 rows x 128 bf16 (two 64-column halves)
 constexpr int kAbKBytes = 64 * 128 * 2;         // 64 keys x 128 d (two halves)
 constexpr int kAbVBytes = 128 * 64 * 2;         // 128 d x 64 keys (one box)
@@ -347,7 +346,6 @@ __global__ void __launch_bounds__(kAbThreads, 1)
     const int jcol = lane & 15;
     const int64_t head_stride = static_cast<int64_t>(a.Nq) * 128;
     int nq = 0;
-    int pend[kAbLag + 1] = {}, np_head = 0, npend = 0;
     auto tile_words = [&](const Stream& st) -> uint32_t {
       if (st.item >= total) return 0u;
       const int p0 = st.inf.y + st.tl * TQ;
@@ -375,30 +373,17 @@ __global__ void __launch_bounds__(kAbThreads, 1)
         const int qi = r / G, hd = r % G;
         const uint32_t wq = __shfl_sync(kFull, twv, qi);
         const uint32_t dst = qd + r * 128 + (((jcol & 7) ^ (r & 7)) << 4);
-        if (wq != 0xffffffffu) {
-          cp16(dst, qg + hd * head_stride + static_cast<int64_t>(wq >> 5) * 128);
-        } else {
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};\n" ::"r"(dst), "r"(0u) : "memory");
-        }
+        // rows of absent queries are zero-filled by the copy itself
+        const bool has = wq != 0xffffffffu;
+        cp16_zfill(dst, has ? qg + hd * head_stride + static_cast<int64_t>(wq >> 5) * 128 : qg, has ? 16 : 0);
       }
-      cp_commit();
-      pend[(np_head + npend) % (kAbLag + 1)] = qs;
-      ++npend;
-      if (npend > kAbLag) {
-        cp_wait<kAbLag>();
-        fence_proxy_async();
-        mbar_arrive(&qfull[pend[np_head]]);
-        np_head = (np_head + 1) % (kAbLag + 1);
-        --npend;
-      }
+      // The stage's barrier completes once every loader thread's copies so
+      // far have landed; the MMA thread fences the async proxy after
+      // observing it.
+      cp_arrive_noinc(&qfull[qs]);
       ++nq;
     }
     cp_wait<0>();
-    fence_proxy_async();
-    for (; npend > 0; --npend) {
-      mbar_arrive(&qfull[pend[np_head]]);
-      np_head = (np_head + 1) % (kAbLag + 1);
-    }
   } else if (warp == kAbMmaWarp) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
@@ -412,17 +397,35 @@ __global__ void __launch_bounds__(kAbThreads, 1)
       // item two back, its stage's last user). S runs in tile order and O in
       // tile order. With no progress for kWaitNs the loop gives up (counted
       // as a fault), like every bounded wait.
-      auto load_kv = [&](int j) {
+      // A K/V request waits in kv_pend[stage] (item j, its record loaded
+      // when the request is made) until the stage's previous O MMAs have
+      // completed; the polling loop issues it then, without blocking.
+      // (Two named registers per stage rather than arrays, so that the
+      // record's load is not waited for until the request is issued.)
+      int kv_pend0 = -1, kv_pend1 = -1;
+      int4 kv_inf0 = make_int4(0, 0, 0, 0), kv_inf1 = make_int4(0, 0, 0, 0);
+      auto request_kv = [&](int j) {
         const int it = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
         if (it >= total) return;
-        const int4 inf = ws.item_info[it];
-        const int kb = j & 1;
-        mbar_wait(&kvempty[kb], ((j >> 1) & 1) ^ 1, faults);
+        if (j & 1) {
+          kv_pend1 = j;
+          kv_inf1 = ws.item_info[it];
+        } else {
+          kv_pend0 = j;
+          kv_inf0 = ws.item_info[it];
+        }
+      };
+      auto try_issue_kv = [&](int kb) -> bool {
+        const int j = kb ? kv_pend1 : kv_pend0;
+        if (j < 0 || !mbar_test(&kvempty[kb], ((j >> 1) & 1) ^ 1)) return false;
+        const int4 inf = kb ? kv_inf1 : kv_inf0;
         const int ky = static_cast<int>(static_cast<int64_t>(inf.x) * a.N + static_cast<int64_t>(inf.w) * 64);
         mbar_expect_tx(&kvfull[kb], kAbKBytes + kAbVBytes);
         tma_load_2d(kbuf + kb * kAbKBytes, &tmk, 0, ky, &kvfull[kb]);
         tma_load_2d(kbuf + kb * kAbKBytes + kAbKBytes / 2, &tmk, 64, ky, &kvfull[kb]);
         tma_load_2d(vbuf + kb * kAbVBytes, &tmvt, inf.w * 64, inf.x * 128, &kvfull[kb]);
+        (kb ? kv_pend1 : kv_pend0) = -1;
+        return true;
       };
       struct Pend {
         int n, j;
@@ -431,8 +434,10 @@ __global__ void __launch_bounds__(kAbThreads, 1)
       constexpr int kF = kAbGroups;  // S issued, O pending: at most one tile per TMEM stage
       Pend fifo[kF];
       int f_head = 0, f_len = 0;
-      load_kv(0);
-      load_kv(1);
+      request_kv(0);
+      request_kv(1);
+      try_issue_kv(0);
+      try_issue_kv(1);
       Stream sm = stream_begin();
       int n = 0, j = -1;
       uint64_t t_prog = global_ns();
@@ -452,11 +457,13 @@ __global__ void __launch_bounds__(kAbThreads, 1)
             --f_len;
             if (pd.last) {
               umma_commit(&kvempty[kb]);
-              load_kv(pd.j + 2);
+              request_kv(pd.j + 2);
             }
             prog = true;
           }
         }
+        if (try_issue_kv(0)) prog = true;
+        if (try_issue_kv(1)) prog = true;
         if (sm.item < total && f_len < kF) {
           const bool first = sm.tl == 0;
           const int jn = first ? j + 1 : j;
@@ -467,6 +474,7 @@ __global__ void __launch_bounds__(kAbThreads, 1)
           ready = ready && mbar_test(&tfree[s], (u & 1) ^ 1);  // the group has read O of tile n - kAbGroups
           if (ready) {
             j = jn;
+            fence_proxy_async();  // the loaders' cp.async writes, before the tensor cores read them
             tc_fence_after();
             const uint32_t qa = smem_u32(qbuf + qs * kAbQBytes), ka = smem_u32(kbuf + (j & 1) * kAbKBytes);
 #pragma unroll

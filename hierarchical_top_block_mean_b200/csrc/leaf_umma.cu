@@ -43,7 +43,6 @@ constexpr int kUmmaThreads = 32 * (kMmaWarp + 1);
 constexpr int kLoaders = 32 * kLoadWarps;
 constexpr int kTilePairs = 16;             // queries per MMA tile (x 8 heads = 128 rows)
 constexpr int kQStages = 5;
-constexpr int kLag = 2;                    // loader publishes a stage kLag tiles after filling it
 constexpr int kQStageBytes = kTilePairs * 8 * 128 * 2;  // 16 queries x 8 heads x 256 B = 32 KB (two 64-col halves)
 constexpr int kKeyBytes = 64 * 128 * 2;                 // 16 KB (two 64-col halves)
 constexpr int kAccCols = 64;                            // fp32 columns per accumulator (N = 64 keys)
@@ -137,7 +136,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     const int g0 = 2 * lw + (lane >> 4);          // head row g0 (and g0 + 4 with two loader warps)
     const int64_t head_stride = static_cast<int64_t>(a.Nq) * 128;
     int nq = 0;                        // uses of the query ring so far
-    int pend[kLag + 1] = {}, np_head = 0, npend = 0;  // filled stages not yet published (FIFO)
     // Each tile's pair words are loaded one tile ahead, so their latency
     // hides behind the previous tile's copies.
     auto tile_words = [&](const Stream& st) -> uint32_t {
@@ -168,38 +166,31 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         mbar_wait(&qempty[qs], ((nq / kQStages) & 1) ^ 1, faults);
         const uint32_t qd = smem_u32(qbuf + qs * kQStageBytes);
         const uint32_t d0 = qd + (jcol >> 3) * (kQStageBytes / 2) + g0 * 128 + (((jcol & 7) ^ g0) << 4);
-        for (int i = 0; i < np; ++i) {
-          const int tq = __shfl_sync(kFull, tw, i);
-          const bf16* src = qrow0 + static_cast<int64_t>(tq) * 128;
-          cp16(d0 + i * 1024, src);
-          if (kLoadWarps == 2) {
-            const uint32_t d1 =
-                qd + (jcol >> 3) * (kQStageBytes / 2) + (g0 + 4) * 128 + (((jcol & 7) ^ (g0 + 4)) << 4);
-            cp16(d1 + i * 1024, src + 4 * head_stride);
+        // Unrolled over the tile's 16 slots so that the shuffles and copies
+        // of different slots overlap instead of forming one chain.
+        int tq[kTilePairs];
+#pragma unroll
+        for (int i = 0; i < kTilePairs; ++i) tq[i] = __shfl_sync(kFull, tw, i);
+#pragma unroll
+        for (int i = 0; i < kTilePairs; ++i) {
+          if (i < np) {
+            const bf16* src = qrow0 + static_cast<int64_t>(tq[i]) * 128;
+            cp16(d0 + i * 1024, src);
+            if (kLoadWarps == 2) {
+              const uint32_t d1 =
+                  qd + (jcol >> 3) * (kQStageBytes / 2) + (g0 + 4) * 128 + (((jcol & 7) ^ (g0 + 4)) << 4);
+              cp16(d1 + i * 1024, src + 4 * head_stride);
+            }
           }
         }
-        cp_commit();
-        // Publish the stage filled kLag tiles ago: its copies have landed
-        // (at most kLag newer groups pending), and the proxy fence makes these
-        // generic-proxy writes visible to the tensor cores' async-proxy reads.
-        pend[(np_head + npend) % (kLag + 1)] = qs;
-        ++npend;
-        if (npend > kLag) {
-          cp_wait<kLag>();
-          fence_proxy_async();
-          mbar_arrive(&qfull[pend[np_head]]);
-          np_head = (np_head + 1) % (kLag + 1);
-          --npend;
-        }
+        // The stage's barrier completes once every loader thread's copies so
+        // far have landed; the MMA thread fences the async proxy after
+        // waiting on it. The loader itself never waits for its copies.
+        cp_arrive_noinc(&qfull[qs]);
         ++nq;
       }
     }
     cp_wait<0>();
-    fence_proxy_async();
-    for (; npend > 0; --npend) {
-      mbar_arrive(&qfull[pend[np_head]]);
-      np_head = (np_head + 1) % (kLag + 1);
-    }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
@@ -227,6 +218,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         for (int tl = 0; tl < c.ntiles; ++tl) {
           const int qs = nq % kQStages;
           mbar_wait(&qfull[qs], (nq / kQStages) & 1, faults);
+          fence_proxy_async();  // the loaders' cp.async writes, before the tensor cores read them
           const int as = na % kAccStages;
           mbar_wait(&accempty[as], ((na / kAccStages) & 1) ^ 1, faults);
           tc_fence_after();

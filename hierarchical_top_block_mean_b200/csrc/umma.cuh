@@ -55,6 +55,17 @@ __device__ inline void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.alig
 __device__ inline void cp16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
 }
+// 16-byte cp.async of src_bytes (16 or 0) bytes, the rest zero-filled
+// (nothing is read when src_bytes is 0).
+__device__ inline void cp16_zfill(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// Arrive on bar once all of this thread's earlier cp.async copies have
+// completed, without adding to the barrier's expected count (the count at
+// init includes this arrival).
+__device__ inline void cp_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
 __device__ inline void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ inline void cp_wait() {
