@@ -713,6 +713,14 @@ def run_gpu(args):
 
     pk, pk_kind = peaks()
     kernels = kernel_rooflines(w, kern_ms, flat_ms, exact_ms, decode, pk, pk_kind)
+    # Measured DRAM bytes per launch (ncu capture in profiles/traffic.json, while the kernel's
+    # sources are unchanged) over this run's time per launch: the kernel's DRAM rate.
+    for name, kr in kernels.items():
+        t = measured_traffic(w.name, name)
+        if t is not None and kr.get("ms"):
+            kr["traffic"] = t
+            kr["dram_gbs"] = t / (kr["ms"] * 1e-3) / 1e9
+            kr["dram_frac"] = kr["dram_gbs"] / pk["hbm_gbs"]
     # Roofline of the dominant kernel of the step (largest share of its time).
     step_kernels = [n for n in kern_ms if n in kernels]
     top = max(step_kernels, key=lambda n: kernels[n]["ms"])
