@@ -68,7 +68,12 @@ size_t carve(const PrefillArgs& a, char* base, Ws* w) {
   x.bucket_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.item_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.pairs = reinterpret_cast<uint32_t*>(take(rows * 32 * 4));
-  x.planes = reinterpret_cast<uint4*>(take(static_cast<size_t>(a.B) * a.H_kv * make_layout(a.N, a.C).R * a.d * 4));
+  const size_t prow = static_cast<size_t>(a.B) * a.H_kv * make_layout(a.N, a.C).R;
+  x.planes = reinterpret_cast<uint4*>(take(prow * a.d * 4));
+  const bool top = router_top_supported(a);
+  x.hi = top ? reinterpret_cast<bf16*>(take(prow * a.d * 2)) : nullptr;
+  x.lo = top ? reinterpret_cast<bf16*>(take(prow * a.d * 2)) : nullptr;
+  x.dense = top ? reinterpret_cast<float*>(take(rows * kDenseSlots * 4)) : nullptr;
   x.item_bucket = reinterpret_cast<int32_t*>(take((rows * 32 / kPairsPerItem + nb + 1) * 4));
   x.item_info = reinterpret_cast<int4*>(take((rows * 32 / kPairsPerItem + nb + 1) * 16));
   x.win_shift = sh;
@@ -81,7 +86,7 @@ size_t carve(const PrefillArgs& a, char* base, Ws* w) {
 // reads ready MMA operands: chunk c of a row holds hi(x[4c..4c+3]) then
 // lo(x[4c..4c+3]), with x - hi - lo below 2^-16 |x|.
 __global__ void __launch_bounds__(256) split_kernel(const float4* __restrict__ pyr, uint4* __restrict__ planes,
-                                                   int64_t n4) {
+                                                   uint2* __restrict__ hi, uint2* __restrict__ lo, int64_t n4) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float4 x = pyr[i];
@@ -90,7 +95,12 @@ __global__ void __launch_bounds__(256) split_kernel(const float4* __restrict__ p
     split_bf16(x.y, h[1], l[1]);
     split_bf16(x.z, h[2], l[2]);
     split_bf16(x.w, h[3], l[3]);
-    planes[i] = make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]));
+    const uint4 v = make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]));
+    planes[i] = v;
+    if (hi) {  // the same parts as plain row-major planes, for the tensor-memory router levels
+      hi[i] = make_uint2(v.x, v.y);
+      lo[i] = make_uint2(v.z, v.w);
+    }
   }
 }
 
@@ -138,6 +148,15 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
       qb[ks][0] = gid < G ? u.x : 0u;
       qb[ks][1] = gid < G ? u.y : 0u;
     }
+    // Levels whose node scores the tensor-memory pass has written: the top
+    // three scored levels of this row's block of kDenseQ queries.
+    int ltop = -1;
+    const float* drow = nullptr;
+    if (ws.dense) {
+      const int64_t last = min(static_cast<int64_t>(a.Nq) - 1, (i_row / kDenseQ) * kDenseQ + kDenseQ - 1);
+      ltop = start_level(n, C, K, a.q0 + last, causal);
+      drow = ws.dense + row * kDenseSlots;
+    }
     // Usable blocks of a level are exactly the first valid_count of them, so
     // one count per level replaces a per-candidate test.
     int vc = static_cast<int>(valid_count(n, C, l, t, causal));
@@ -145,7 +164,13 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
       const int vcc = static_cast<int>(valid_count(n, C, l - 1, t, causal));  // usable children level
       const int nc = warp_compact(cand, cand >= 0 && cand < vc, tmp[warp]);
       int nk = nc;
-      if (nc > K) {
+      if (nc > K && l <= ltop && l >= ltop - 2) {
+        float s = lane < nc ? __ldg(drow + dense_slot0(ltop - l) + cand) : -INFINITY;
+        int idx = lane < nc ? cand : INT_MAX;
+        warp_sort_desc(s, idx);
+        cand = idx;
+        nk = K;
+      } else if (nc > K) {
         // M-tile m holds candidates 8m .. 8m+7: row gid = first child, row gid + 8 = second.
         float um[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -587,10 +612,12 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
     const int64_t gb = (n4 + 255) / 256;
     const unsigned g = static_cast<unsigned>(gb < sm_count() * 16 ? gb : sm_count() * 16);
     TimedLaunch tl("split_kernel", st);
-    split_kernel<<<g, 256, 0, st>>>(reinterpret_cast<const float4*>(pyr), ws.planes, n4);
+    split_kernel<<<g, 256, 0, st>>>(reinterpret_cast<const float4*>(pyr), ws.planes, reinterpret_cast<uint2*>(ws.hi),
+                                    reinterpret_cast<uint2*>(ws.lo), n4);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (ws.dense && (e = launch_router_top(a, q, lay, ws, st)) != cudaSuccess) return e;
   e = dispatch_tdg(PISA_DTYPE_BF16, a.d, G, [&](auto, auto dd, auto gg) -> cudaError_t {
     constexpr int D = decltype(dd)::value, GG = decltype(gg)::value;
     TimedLaunch tl("router_kernel", st);

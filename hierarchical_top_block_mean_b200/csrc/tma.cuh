@@ -23,6 +23,11 @@ cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols,
 // 64 x box1 x box2 elements and 128-byte swizzle.
 cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                               uint32_t box1, uint32_t box2);
+// 3-D bf16 map with explicit byte strides of dimensions 1 and 2 (any order of
+// magnitude, e.g. a head dimension outside a token dimension), a box of
+// 64 x box1 x box2 elements and 128-byte swizzle.
+cudaError_t make_tmap_bf16_3d_strided(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                                      uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1, uint32_t box2);
 
 // Device address of the fault counter (bounded waits that ran out) on the
 // current device; kernels that wait take it as an argument.
