@@ -166,7 +166,9 @@ def work_model(w):
     geometry alone (one pass over every query position t):
       router: per query row and scored inner level l >= 2, up to 2K
         candidates, each gathering its <= 2 child summaries (d fp32 values,
-        stored as bf16 hi + lo) from L2;
+        stored as bf16 hi + lo) from L2, except on the levels the tensor-core
+        pass scores (router_top_flops: 2 x 2 x 128 x d per child row of a
+        16-query block's top three levels, hi and lo);
       leaf scorer: (query, candidate leaf) pairs at the leaf level, each
         2 G_Q C d flops;
       attention: 4 G_Q d flops per usable key of the K selected blocks;
@@ -177,14 +179,34 @@ def work_model(w):
     L = api.pyramid_geometry(w.N, w.C)[0]
     K, G, e = w.K, w.H_q // w.H_kv, (2 if w.dtype == "bf16" else 4)
     heads = w.B * w.H_kv
+    # Levels scored on tensor cores for G_Q = 8, d = 128 (bf16, K <= 16, C a
+    # power of two): the top three scored levels of each block of 16 queries,
+    # taken at the block's last query; those levels are read, not gathered.
+    dense = (w.dtype == "bf16" and w.d == 128 and G == 8 and K <= 16 and (w.C & (w.C - 1)) == 0)
+    last = np.minimum(w.N - 1, (t // 16) * 16 + 15)
+    ltop = np.zeros(w.N, dtype=np.int64)
+    for l in range(L, 0, -1):
+        ltop = np.where((ltop == 0) & (_valid(w, l, last) > K), l, ltop)
     gathered = np.zeros(w.N)
     started = np.zeros(w.N, dtype=bool)
     for l in range(L, 1, -1):
         v = _valid(w, l, t)
         scored = started | (v > K)
         cand = np.where(started, np.minimum(2 * K, v), v)
-        gathered += np.where(scored, cand * 2, 0)
+        in_dense = dense & (l <= ltop) & (l >= ltop - 2)
+        gathered += np.where(scored & ~in_dense, cand * 2, 0)
         started = scored
+    # Children rows the tensor-core levels multiply per block (hi and lo parts).
+    top_rows = 0.0
+    if dense:
+        blocks_last = last[::16]
+        for i in range(3):
+            lb = ltop[::16] - i
+            ok = lb >= 2
+            for l in np.unique(lb[ok]):
+                sel = ok & (lb == l)
+                size_below = -(-w.N // (w.C << (int(l) - 2)))
+                top_rows += np.minimum(2 * _valid(w, int(l), blocks_last[sel]), size_below).sum()
     v1 = _valid(w, 1, t)
     pairs = np.where(v1 > K, np.where(started, np.minimum(2 * K, v1), v1), 0)
     keys = np.minimum(K * w.C, t + 1) if w.causal else np.full(w.N, min(K * w.C, w.N))
@@ -201,6 +223,7 @@ def work_model(w):
         "attn_partial_bytes": heads * w.N * K * G * (128 * 2 + 8),
         "attn_out_bytes": w.B * w.H_q * w.N * (w.d * e + 4),
         "split_bytes": heads * api.pyramid_rows(w.N, w.C) * w.d * 8,
+        "router_top_flops": heads * top_rows * 2 * 2 * 128 * w.d,
     }.items()}
 
 
@@ -298,6 +321,9 @@ def kernel_rooflines(w, kern, flat_ms, exact_ms, decode, pk, pk_kind):
     add("pyramid_kernel", *k("pyramid_kernel"), "hbm", pyramid_bytes(w),
         "keys read once + fp32 pyramid written once (one cooperative launch)")
     add("split_kernel", *k("split_kernel"), "hbm", m["split_bytes"], "fp32 pyramid read, bf16 hi/lo planes written")
+    add("router_top_kernel", *k("router_top_kernel"), "tensor", m["router_top_flops"],
+        "hi and lo products of 128 (query, head) rows with the children of the top three scored levels of each "
+        "16-query block")
     r = k("router_kernel")
     if r[0]:
         add("router_kernel", *r, "hbm", m["router_hbm_bytes"],
