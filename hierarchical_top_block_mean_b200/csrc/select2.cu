@@ -1,8 +1,12 @@
 // Two-stage PISA selection for bf16 inputs (paper §Kernels, training and
 // prefill kernels):
-//   stage 1  router_kernel     one warp per (kv head, query): levels L..2 of
-//                              the coarse-to-fine search; candidate children
-//                              scored on tensor cores.
+//   stage 1  router_top_kernel (router_top.cu; G_Q = 8, d = 128) every node
+//                              of the top three scored levels of each block
+//                              of 16 queries, on tcgen05;
+//            router_kernel     one warp per (kv head, query): levels L..2 of
+//                              the coarse-to-fine search, reading those node
+//                              scores where present, else scoring the
+//                              candidates' children on tensor cores.
 //   grouping count (in stage 1), scan_kernel, scatter_kernel,
 //                              itemize_kernel: a CSR of the (query, candidate
 //                              leaf) pairs keyed by (kv head, query window,
