@@ -5,7 +5,7 @@
 //
 // One CTA per SM runs a warp-specialised pipeline over the stage-2 work
 // items (64 (query, leaf) pairs of one bucket, walked grid-strided so that
-// all SMs share the current query window in L2):
+// all SMs work in the current query window):
 //   warps 8-11 (loads): per tile of 16 queries, their 8 head rows
 //     (16 x 8 = 128 rows) gathered with 16-byte cp.async straight into the
 //     swizzled operand layout of a ring of query stages, running ahead of the
