@@ -10,7 +10,7 @@
 //   grouping count (in stage 1), scan_kernel, scatter_kernel,
 //                              itemize_kernel: a CSR of the (query, candidate
 //                              leaf) pairs keyed by (kv head, query window,
-//                              leaf), cut into work items of 64 pairs.
+//                              leaf), cut into work items of 128 pairs.
 //   stage 2  leaf_umma_kernel  (leaf_umma.cu; G_Q = 8, d = 128, C = 64) or
 //            leaf_kernel       per work item: the C x d key tile is brought
 //                              into shared memory once and reused across
@@ -36,7 +36,7 @@ namespace pisa {
 namespace {
 
 constexpr int kRouterWarps = 4;
-constexpr int kPairsPerItem = 64;  // stage-2 work item: 16 query tiles of Q_tile = 4 pairs
+constexpr int kPairsPerItem = 128;  // stage-2 work item (64 measured 6 % slower at 256K: more key-tile loads)
 constexpr int kQTile = 4;
 constexpr int kLeafThreads = 256;
 
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(256) itemize_kernel(Ws ws, int nb, int M1) {
 }
 
 // ---------------------------------------------------------------- stage 2
-// Stage 2. Work items (64 pairs of one bucket) are walked grid-strided, so
+// Stage 2. Work items (128 pairs of one bucket) are walked grid-strided, so
 // that at any time all CTAs work on neighbouring buckets (the same query
 // window). Per item the leaf's C x d key
 // tile is brought into shared memory by bulk tensor copies (double buffered
