@@ -71,7 +71,7 @@ constexpr uint32_t kIdescO = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) <
 
 struct AbWs {
   int32_t* count;       // [nb] pairs per bucket
-  int32_t* fill;        // [nb] scatter cursors
+  int32_t* rank;        // [rows K] each selected (row, slot) entry's position in its bucket
   int32_t* off;         // [nb + 1] bucket offsets
   int32_t* item_off;    // [nb + 1] item offsets
   uint32_t* pairs;      // [rows K] (query row << 5 | slot), grouped by bucket
@@ -114,7 +114,7 @@ size_t ab_carve(const PrefillArgs& a, char* base, AbWs* w) {
   };
   AbWs x;
   x.count = reinterpret_cast<int32_t*>(take(nb * 4));
-  x.fill = reinterpret_cast<int32_t*>(take(nb * 4));
+  x.rank = reinterpret_cast<int32_t*>(take(rows * a.K * 4));
   x.off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.item_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.pairs = reinterpret_cast<uint32_t*>(take(rows * a.K * 4));
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(256) attn_count_kernel(const int32_t* __restri
     const int leaf = sel[x];
     if (leaf < 0 || leaf >= M1) continue;
     const int64_t row = x / K;
-    atomicAdd(&w.count[ab_bucket(w, row / Nq, row % Nq, M1, leaf)], 1);
+    w.rank[x] = atomicAdd(&w.count[ab_bucket(w, row / Nq, row % Nq, M1, leaf)], 1);  // place in the bucket
   }
 }
 
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(256) attn_scatter_kernel(const int32_t* __rest
     const int slot = static_cast<int>(x % K);
     const int64_t i_row = row % Nq;
     const int64_t b = ab_bucket(w, row / Nq, i_row, M1, leaf);
-    const int pos = atomicAdd(&w.fill[b], 1);
+    const int pos = w.rank[x];
     w.pairs[w.off[b] + pos] = (static_cast<uint32_t>(i_row) << 5) | static_cast<uint32_t>(slot);
   }
 }
@@ -760,7 +760,6 @@ cudaError_t launch_attn_bucket(const PrefillArgs& a, const void* q, const void* 
   const int nb = static_cast<int>(static_cast<int64_t>(a.B) * a.H_kv * w.nwin * M1);
   const int64_t entries = rows * a.K;
   cudaError_t e = cudaMemsetAsync(w.count, 0, static_cast<size_t>(nb) * 4, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(w.fill, 0, static_cast<size_t>(nb) * 4, st);
   if (e != cudaSuccess) return e;
   const int sms = ab_sm_count();
   const unsigned eg = static_cast<unsigned>(std::min<int64_t>((entries + 255) / 256, static_cast<int64_t>(sms) * 32));

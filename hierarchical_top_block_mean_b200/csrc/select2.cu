@@ -72,7 +72,7 @@ size_t carve(const PrefillArgs& a, char* base, Ws* w) {
   x.ncand = reinterpret_cast<int32_t*>(take(rows * 4));
   x.score = reinterpret_cast<float*>(take(rows * 32 * 4));
   x.count = reinterpret_cast<int32_t*>(take(nb * 4));
-  x.fill = reinterpret_cast<int32_t*>(take(nb * 4));
+  x.rank = reinterpret_cast<int32_t*>(take(rows * 32 * 4));
   x.bucket_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.item_off = reinterpret_cast<int32_t*>(take((nb + 1) * 4));
   x.pairs = reinterpret_cast<uint32_t*>(take(rows * 32 * 4));
@@ -253,7 +253,10 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
   }
   ws.cand[row * 32 + lane] = lane < nc ? cand : -1;
   if (lane == 0) ws.ncand[row] = nc;
-  if (lane < nc) atomicAdd(&ws.count[(bh * ws.nwin + (i_row >> ws.win_shift)) * level_size(n, C, 1) + cand], 1);
+  // The count's old value is the pair's place in its bucket, so the scatter
+  // needs no second atomic.
+  if (lane < nc)
+    ws.rank[row * 32 + lane] = atomicAdd(&ws.count[(bh * ws.nwin + (i_row >> ws.win_shift)) * level_size(n, C, 1) + cand], 1);
 }
 
 // ---------------------------------------------------------------- grouping
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(Ws ws, int64_t rows, int N
   const int leaf = ws.cand[row * 32 + slot];
   const int64_t bh = row / Nq, t = row % Nq;
   const int64_t bucket = (bh * ws.nwin + (t >> ws.win_shift)) * M1 + leaf;
-  const int pos = atomicAdd(&ws.fill[bucket], 1);
+  const int pos = ws.rank[row * 32 + slot];
   ws.pairs[ws.bucket_off[bucket] + pos] = (static_cast<uint32_t>(t) << 5) | static_cast<uint32_t>(slot);
 }
 
@@ -612,7 +615,6 @@ cudaError_t launch_select2(const PrefillArgs& a, const void* q, const void* k, c
   const int M1 = static_cast<int>(level_size(a.N, a.C, 1));
   const int nb = a.B * a.H_kv * ws.nwin * M1;
   cudaError_t e = cudaMemsetAsync(ws.count, 0, static_cast<size_t>(nb) * 4, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ws.fill, 0, static_cast<size_t>(nb) * 4, st);
   if (e != cudaSuccess) return e;
   const int G = a.H_q / a.H_kv;
   {

@@ -11,7 +11,7 @@ struct Ws {
   int32_t* ncand;       // [rows] candidates per row; -1 when stage 1 already wrote sel
   float* score;         // [rows][32] leaf score of each candidate slot
   int32_t* count;       // [buckets] pairs per (b, kv head, leaf)
-  int32_t* fill;        // [buckets] scatter cursors
+  int32_t* rank;        // [rows][32] each candidate's position in its bucket (its count's old value)
   int32_t* bucket_off;  // [buckets + 1] exclusive scan of count
   int32_t* item_off;    // [buckets + 1] exclusive scan of ceil(count / kPairsPerItem)
   uint32_t* pairs;      // [rows * 32] (query row << 5 | slot), grouped by bucket
