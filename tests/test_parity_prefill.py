@@ -27,6 +27,11 @@ SMALL = [
                                                  K=8, dtype="bf16", seed=1300),
     workloads.PREFILL["tiny_noncausal_1k"].with_(name="bf16_G2_B2", B=2, N=777, H_q=4, H_kv=2, d=64, C=32, K=3,
                                                  causal=True, dtype="bf16", seed=1400),
+    # G_Q = 8, d = 128 with two sequences and three kv heads: the tensor-core
+    # router levels, the tcgen05 leaf scorer and the bucketed attention index
+    # batch and head together; a ragged last query block.
+    workloads.PREFILL["clustered_64k"].with_(name="clustered_3k_G8_B2_H3", B=2, N=3001, H_q=24, H_kv=3,
+                                             segment=384, seed=3300),
 ]
 
 
