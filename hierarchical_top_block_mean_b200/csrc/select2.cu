@@ -580,12 +580,47 @@ __global__ void __launch_bounds__(256) final_kernel(PrefillArgs a, Ws ws, int32_
   if (nc < 0) return;  // stage 1 kept every usable leaf unscored and wrote sel
   float s = lane < nc ? ws.score[row * 32 + lane] : -INFINITY;
   int idx = lane < nc ? ws.cand[row * 32 + lane] : INT_MAX;
-  warp_sort_desc(s, idx);
+  // Top K (K <= 16) by (score descending, index ascending): the first four
+  // phases of a 32-lane bitonic sort order lanes 0..15 best-first and lanes
+  // 16..31 worst-first; keeping the better of lanes i and i + 16 leaves the 16
+  // best in lanes 0..15. Only for K < 16 are those 16 then ordered, so that
+  // lanes 0..K-1 hold the K best.
+  auto cmpx = [&](int j, bool keep_best) {
+    const float os = __shfl_xor_sync(kFull, s, j);
+    const int oi = __shfl_xor_sync(kFull, idx, j);
+    if (keep_best ? ranks_before(os, oi, s, idx) : ranks_before(s, idx, os, oi)) {
+      s = os;
+      idx = oi;
+    }
+  };
+#pragma unroll
+  for (int k = 2; k <= 16; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) cmpx(j, ((lane & k) == 0) == ((lane & j) == 0));
+  cmpx(16, (lane & 16) == 0);
+  if (a.K < 16) {
+#pragma unroll
+    for (int j = 8; j > 0; j >>= 1) cmpx(j, (lane & j) == 0);
+  }
   if (lane >= a.K) {
     idx = INT_MAX;
     s = 0.f;
   }
-  warp_sort_asc_kv(idx, s);
+  // The K kept pairs ascending by index: a 16-lane bitonic sort (lanes 16..31
+  // hold only empty slots and take no part).
+#pragma unroll
+  for (int k = 2; k <= 16; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const int oi = __shfl_xor_sync(kFull, idx, j);
+      const float os = __shfl_xor_sync(kFull, s, j);
+      const bool keep_small = ((lane & k) == 0) == ((lane & j) == 0);
+      if (keep_small ? (oi < idx) : (oi > idx)) {
+        idx = oi;
+        s = os;
+      }
+    }
+  }
   if (lane < a.K) {
     sel[row * a.K + lane] = idx;
     if (sel_score) sel_score[row * a.K + lane] = s;
