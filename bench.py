@@ -96,11 +96,27 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return self
+        # nvidia-smi takes a few hundred ms to start; a timed region of a few
+        # hundred ms would otherwise end before its first sample. Wait (up to
+        # 5 s) for the first sample, and count the samples taken before the
+        # region so that the summary can leave them out.
+        t_end = time.time() + 5.0
+        while time.time() < t_end and self.proc.poll() is None and self._lines() == 0:
+            time.sleep(0.02)
+        self.before = self._lines()
         return self
+
+    def _lines(self):
+        try:
+            with open(self.path) as f:
+                return sum(1 for line in f if line.strip())
+        except OSError:
+            return 0
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -117,20 +133,25 @@ class ClockSampler:
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
+            lines = [line for line in f if line.strip()]
+        # Samples taken during the region; the last one taken just before it
+        # stands in only when the region was shorter than the sampling period.
+        during = lines[getattr(self, "before", 0):]
+        for line in (during if during else lines[-1:]):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "sampled": "during the timed region" if during else "just before the timed region"}
 
 
 def events(n):
