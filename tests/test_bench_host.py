@@ -85,3 +85,53 @@ def test_work_model_matches_the_oracle_trace(oracle):
     assert pairs <= m["leaf_pairs"] <= 1.05 * pairs
     assert m["leaf_flops"] == m["leaf_pairs"] * 2 * (w.H_q // w.H_kv) * w.C * w.d
     assert gathered * w.d * 4 <= m["router_gather_bytes"] <= 1.10 * gathered * w.d * 4
+
+
+def test_work_model_leaves_out_the_tensor_core_router_levels():
+    """At G_Q = 8, d = 128 (bf16) the router reads the node scores of each
+    16-query block's top three scored levels (taken at the block's last query)
+    instead of gathering children. The work model must count gathers only on
+    the other scored levels, and the tensor-core pass's children rows on
+    those three. Checked against a per-position loop over the level geometry."""
+    from hierarchical_top_block_mean_b200 import workloads
+    w = workloads.Prefill("model_g8", B=1, N=5000, H_q=8, H_kv=1, d=128, C=64, K=16, causal=True, dtype="bf16",
+                          seed=3)
+    m = bench.work_model(w)
+    L = 1
+    while -(-w.N // (w.C << (L - 1))) > 1:
+        L += 1
+    size = {l: -(-w.N // (w.C << (l - 1))) for l in range(1, L + 1)}
+
+    def valid(l, t):
+        return min(size[l], t // (w.C << (l - 1)) + 1)
+
+    def start(t):
+        l = L
+        while l >= 1 and valid(l, t) <= w.K:
+            l -= 1
+        return l
+
+    gathered = 0
+    for t in range(w.N):
+        top = start(min(w.N - 1, (t // 16) * 16 + 15))
+        started = False
+        for l in range(L, 1, -1):
+            v = valid(l, t)
+            scored = started or v > w.K
+            if scored and not (top - 2 <= l <= top):
+                gathered += 2 * (min(2 * w.K, v) if started else v)
+            started = scored
+    rows = 0
+    for blk in range(-(-w.N // 16)):
+        last = min(w.N - 1, blk * 16 + 15)
+        top = start(last)
+        for i in range(3):
+            l = top - i
+            if l < 2:
+                break
+            rows += min(2 * valid(l, last), size[l - 1])
+    assert m["router_gather_bytes"] == gathered * w.d * 4
+    assert m["router_top_flops"] == rows * 2 * 2 * 128 * w.d
+    # and with the tensor-core pass off (f32), every scored level is gathered
+    m32 = bench.work_model(w.with_(dtype="f32"))
+    assert m32["router_top_flops"] == 0 and m32["router_gather_bytes"] > m["router_gather_bytes"]
