@@ -135,3 +135,25 @@ def test_work_model_leaves_out_the_tensor_core_router_levels():
     # and with the tensor-core pass off (f32), every scored level is gathered
     m32 = bench.work_model(w.with_(dtype="f32"))
     assert m32["router_top_flops"] == 0 and m32["router_gather_bytes"] > m["router_gather_bytes"]
+
+
+def test_clock_sampler_covers_a_short_timed_region(tmp_path, monkeypatch):
+    """nvidia-smi takes a while to start; the sampler must wait for its first
+    sample so that a timed region shorter than that still gets samples, and it
+    must report only the samples taken during the region. A fake nvidia-smi on
+    PATH (0.3 s start-up, a sample every 50 ms) stands in for the real one."""
+    import os
+    import time
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\nsleep 0.3\nwhile true; do\n"
+                    "  echo '0, 1965, 1965, 500.0, 0x4, Not Active, Not Active, Not Active, Active'\n"
+                    "  sleep 0.05\ndone\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ.get("PATH", ""))
+    with bench.ClockSampler(0) as clk:
+        time.sleep(0.2)  # the timed region
+    s = clk.summary()
+    assert s["sampled"] == "during the timed region"
+    assert s["samples"] >= 1
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
