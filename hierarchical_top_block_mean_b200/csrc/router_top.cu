@@ -106,8 +106,9 @@ __device__ inline int n_chunks_total(const TopGeom& g) {
 __device__ inline int chunk_level(int j) { return j < 2 ? j : 2; }
 __device__ inline int chunk_col(int j) { return j < 2 ? kTopChunkRows * j : 256 + kTopChunkRows * (j - 2); }
 
-// 2^x and log2 x by the hardware's approximate instructions (relative error
-// near 2^-22).
+// 2^x and log2 x by the hardware's approximate instructions (errors near
+// 2^-22: relative for 2^x, absolute for log2 x, whose argument here is a
+// product of eight factors in [1, 2]).
 __device__ inline float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
