@@ -200,10 +200,10 @@ def work_model(w):
     L = api.pyramid_geometry(w.N, w.C)[0]
     K, G, e = w.K, w.H_q // w.H_kv, (2 if w.dtype == "bf16" else 4)
     heads = w.B * w.H_kv
-    # Levels scored on tensor cores for G_Q = 8, d = 128 (bf16, K <= 16, C a
-    # power of two): the top three scored levels of each block of 16 queries,
+    # Levels scored on tensor cores for G_Q = 8, d = 128 (bf16, K <= 16, C =
+    # 64): the top three scored levels of each block of 16 queries,
     # taken at the block's last query; those levels are read, not gathered.
-    dense = (w.dtype == "bf16" and w.d == 128 and G == 8 and K <= 16 and (w.C & (w.C - 1)) == 0)
+    dense = (w.dtype == "bf16" and w.d == 128 and G == 8 and K <= 16 and w.C == 64)
     last = np.minimum(w.N - 1, (t // 16) * 16 + 15)
     ltop = np.zeros(w.N, dtype=np.int64)
     for l in range(L, 0, -1):
